@@ -1,0 +1,198 @@
+"""CPU oracle of the DeepSeek Sparse Attention (DSA) hot path.
+
+TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the benchmark's CPU-baseline leg
+may import this module; the library never calls it and shares no code with it.
+
+Plain, slow and written to be checked by eye against the formulas on the pages, in float64,
+from the FP8 / bf16 storage codes (decoded here by this module's own routines). Positions are
+0-based: the pages' C_t = {1..t} becomes j in [0, p].
+
+Sources ("page" = title of the web page):
+  [P5-LI]  "DeepSeek Sparse Attention：从 SWA 到稀疏 Attention 计算", section "Lightning Indexer：为
+           历史位置打分并选出 top-k": I_tj = sum_r w_tr ReLU(q_tr . k_j) over visible j <= t; one
+           shared key per position; S_t = TopK_{j<=t}(I_tj, k); S_t shared by all attention heads;
+           worked example t=8, k=3 -> S_8 = {2,5,8}.
+  [P5-SA]  same page, section "Sparse Attention：在选中位置上计算 Attention": softmax(QK^T/sqrt(d_h)
+           + M^DSA) V with M = 0 on S_t and -inf elsewhere, computed by reading only the rows in S_t.
+  [P5-SWA] same page, section "SWA：让固定窗口沿序列移动": causal visibility C_t = {1..t}.
+  [P1-DSA] "MTP 与稀疏注意力：NSA 与 DSA", section "稀疏注意力：NSA 与 DSA": 64 FP8 indexer heads of
+           width 128, top 2048, absorbed MLA over a 576-wide latent (512 + 64 rope), per-pair FLOP
+           counts; expanded head width 128 + 64 = 192; k = min(L, 2048).
+
+Readings where the pages leave a step open (each is listed in the design notes):
+  * FP8 is OCP e4m3fn; per-token fp32 scales multiply the decoded codes (s^q_t for the query,
+    s^k_j for the key). Positive scales pass through ReLU unchanged.
+  * Query i of request b (m_b queries, n_b cached positions including them) sits at position
+    p = n_b - m_b + i and sees j in [0, p] (self included).
+  * TopK ties: higher score first, then smaller j. If p+1 <= k every visible position is selected.
+  * Softmax scale tau = 1/sqrt(192) (expanded head width); V = first 512 latent dims.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+PAGE = 64
+D_V = 512
+
+
+# ---------------------------------------------------------------------------------------------
+# storage decoders
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Decode OCP FP8 E4M3 (e4m3fn) codes to float64.
+
+    Bit layout s.eeee.mmm, exponent bias 7. Exponent field 0 gives subnormals (m/8)*2^-6;
+    otherwise (1 + m/8)*2^(e-7). There are no infinities; s.1111.111 is NaN.
+    """
+    c = np.asarray(codes).astype(np.uint8).astype(np.int64)
+    sign = np.where((c & 0x80) != 0, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    mant = (c & 0x7).astype(np.float64)
+    normal = (1.0 + mant / 8.0) * np.exp2(e.astype(np.float64) - 7.0)
+    subnormal = (mant / 8.0) * 2.0 ** -6
+    v = sign * np.where(e == 0, subnormal, normal)
+    return np.where((e == 15) & ((c & 0x7) == 7), np.nan, v)
+
+
+def bf16_decode(bits) -> np.ndarray:
+    """Decode bf16 bit patterns (the upper half of an IEEE float32) to float64."""
+    b = np.asarray(bits).astype(np.uint16).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32).astype(np.float64)
+
+
+# ---------------------------------------------------------------------------------------------
+# batch geometry
+
+def query_positions(seq_lens, cu_q):
+    """(request b, position p) of every query row; query i of request b sits at n_b - m_b + i."""
+    seq_lens = np.asarray(seq_lens, np.int64)
+    cu_q = np.asarray(cu_q, np.int64)
+    T = int(cu_q[-1]) if len(cu_q) else 0
+    req = np.zeros(T, np.int64)
+    pos = np.zeros(T, np.int64)
+    for b in range(len(seq_lens)):
+        m = int(cu_q[b + 1] - cu_q[b])
+        for i in range(m):
+            req[cu_q[b] + i] = b
+            pos[cu_q[b] + i] = int(seq_lens[b]) - m + i
+    return req, pos
+
+
+def physical_rows(block_table_row, positions):
+    """(page, slot) holding logical positions of one request: page = table[j // 64], slot = j % 64."""
+    positions = np.asarray(positions, np.int64)
+    pages = np.asarray(block_table_row, np.int64)[positions // PAGE]
+    return pages, positions % PAGE
+
+
+# ---------------------------------------------------------------------------------------------
+# step 1: Lightning-Indexer scores  [P5-LI], FP8 per [P1-DSA]
+
+def index_scores_row(t, req, pos, block_table, qI, qI_scale, wI, kI_cache, kI_scale) -> np.ndarray:
+    """I_t = [I_t0 .. I_tp] for query row t, float64.
+
+    I_tj = sum_r w_tr * ReLU( (s^q_t q_tr) . (s^k_j k_j) ).
+    """
+    b, p = int(req[t]), int(pos[t])
+    pages, slots = physical_rows(block_table[b], np.arange(p + 1))
+    k = e4m3_decode(kI_cache[pages, slots]) * np.asarray(kI_scale, np.float64)[pages, slots][:, None]
+    qt = e4m3_decode(qI[t]) * float(qI_scale[t])            # [nhI, 128]
+    logits = qt @ k.T                                        # [nhI, p+1]: q_tr . k_j
+    return np.asarray(wI[t], np.float64) @ np.maximum(logits, 0.0)
+
+
+def index_scores(seq_lens, cu_q, block_table, qI, qI_scale, wI, kI_cache, kI_scale, ld=None, rows=None):
+    """Score matrix [T, ld] (float64); -inf at j > p (never visible). `rows` limits the work."""
+    req, pos = query_positions(seq_lens, cu_q)
+    T = len(req)
+    if ld is None:
+        ld = int(np.max(seq_lens)) if len(seq_lens) else 0
+    out = np.full((T, ld), -np.inf)
+    for t in (range(T) if rows is None else rows):
+        out[t, : int(pos[t]) + 1] = index_scores_row(t, req, pos, block_table, qI, qI_scale, wI,
+                                                     kI_cache, kI_scale)
+    return out
+
+
+# ---------------------------------------------------------------------------------------------
+# step 2: TopK  [P5-LI]; k = min(L, TOPK) per [P1-DSA]
+
+def topk_select(scores_row, k) -> np.ndarray:
+    """S_t as int32[k]: positions of the min(k, L) largest scores (ties: smaller j first),
+    in descending score order, padded with -1. `scores_row` holds exactly the L visible scores."""
+    s = np.asarray(scores_row)
+    L = s.shape[0]
+    order = np.lexsort((np.arange(L), -s.astype(np.float64)))   # by -I, then by j
+    out = np.full(k, -1, np.int32)
+    take = min(k, L)
+    out[:take] = np.asarray(order[:take], np.int32)
+    return out
+
+
+def topk(scores, pos, k, rows=None) -> np.ndarray:
+    """Index sets for every row of a score matrix; row t sees its first pos[t]+1 columns."""
+    T = scores.shape[0]
+    out = np.full((T, k), -1, np.int32)
+    for t in (range(T) if rows is None else rows):
+        out[t] = topk_select(scores[t, : int(pos[t]) + 1], k)
+    return out
+
+
+# ---------------------------------------------------------------------------------------------
+# step 3: sparse MLA on S_t  [P5-SA]; absorbed MLA form per [P1-DSA]
+
+def sparse_mla_row(t, req, S_t, block_table, q, kv_cache, softmax_scale):
+    """Attention of query row t over the latent rows in S_t (entries < 0 are padding).
+
+    z_hj = tau * q_th . c_j (576 dims); o_th = sum_j softmax_j(z_hj) c_j[0:512];
+    lse_th = log sum_j exp(z_hj). Returns (o [H, 512], lse [H]) in float64.
+    """
+    b = int(req[t])
+    sel = np.asarray([j for j in S_t if j >= 0], np.int64)
+    qt = bf16_decode(q[t])                                    # [H, 576]
+    H = qt.shape[0]
+    if sel.size == 0:
+        return np.zeros((H, D_V)), np.full(H, -np.inf)
+    pages, slots = physical_rows(block_table[b], sel)
+    c = bf16_decode(kv_cache[pages, slots])                   # [|S_t|, 576]
+    z = softmax_scale * (qt @ c.T)                            # [H, |S_t|]
+    zmax = z.max(axis=1, keepdims=True)
+    e = np.exp(z - zmax)
+    denom = e.sum(axis=1, keepdims=True)
+    o = (e @ c[:, :D_V]) / denom
+    lse = zmax[:, 0] + np.log(denom[:, 0])
+    return o, lse
+
+
+def sparse_mla(seq_lens, cu_q, block_table, q, kv_cache, S, softmax_scale, rows=None):
+    """Output [T, H, 512] and lse [T, H] (float64) for every (or the given) query row."""
+    req, _ = query_positions(seq_lens, cu_q)
+    T, H = q.shape[0], q.shape[1]
+    out = np.zeros((T, H, D_V))
+    lse = np.full((T, H), -np.inf)
+    for t in (range(T) if rows is None else rows):
+        out[t], lse[t] = sparse_mla_row(t, req, S[t], block_table, q, kv_cache, softmax_scale)
+    return out, lse
+
+
+# ---------------------------------------------------------------------------------------------
+# the whole path
+
+def dsa_layer(seq_lens, cu_q, block_table, qI, qI_scale, wI, kI_cache, kI_scale, q, kv_cache,
+              k, softmax_scale, rows=None):
+    """Indexer -> TopK -> sparse MLA for every (or the given) query row.
+
+    Returns dict(scores [T, ld] f64, S [T, k] int32, out [T, H, 512] f64, lse [T, H] f64).
+    """
+    _, pos = query_positions(seq_lens, cu_q)
+    scores = index_scores(seq_lens, cu_q, block_table, qI, qI_scale, wI, kI_cache, kI_scale, rows=rows)
+    S = topk(scores, pos, k, rows=rows)
+    out, lse = sparse_mla(seq_lens, cu_q, block_table, q, kv_cache, S, softmax_scale, rows=rows)
+    return dict(scores=scores, S=S, out=out, lse=lse)
+
+
+def default_softmax_scale() -> float:
+    """tau = 1/sqrt(d_h) with the expanded head width d_h = 128 + 64 = 192 [P1-DSA], [P5-SA]."""
+    return 1.0 / math.sqrt(128 + 64)

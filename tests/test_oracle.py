@@ -1,0 +1,336 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix (no GPU needed).
+
+Each check is chosen so that a plausible slip in the oracle fails it: a dropped ReLU or scale,
+a wrong sign, an off-by-one in the causal set, a wrong page lookup, a transposed operand in the
+attention, a wrong softmax scale or value width, a wrong tie rule.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import dsa_oracle as O
+from oracle import cost_model as CM
+from sparse_attention_12_b200 import synth
+
+
+# ---------------------------------------------------------------------------------------------
+# storage decoders against torch's own conversions
+
+def test_e4m3_decode_matches_torch_all_codes():
+    codes = np.arange(256, dtype=np.uint8)
+    ours = O.e4m3_decode(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], ref[~nan])
+    # anchors from the OCP e4m3 definition
+    assert O.e4m3_decode(np.uint8(0x7E)) == 448.0
+    assert O.e4m3_decode(np.uint8(0x01)) == 2.0 ** -9
+    assert O.e4m3_decode(np.uint8(0x08)) == 2.0 ** -6
+    assert O.e4m3_decode(np.uint8(0x38)) == 1.0
+    assert O.e4m3_decode(np.uint8(0xB8)) == -1.0
+
+
+def test_bf16_decode_matches_torch():
+    rng = np.random.default_rng(1)
+    bits = rng.integers(0, 1 << 16, size=4096, dtype=np.uint16)
+    ours = O.bf16_decode(bits)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], ref[~nan])
+
+
+# ---------------------------------------------------------------------------------------------
+# indexer scores
+
+def _hand_case(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "indexer_hand.json")))
+    code = {float(k): v for k, v in g["e4m3_codes"].items()}
+    P = 8
+    kI = np.zeros((P, 64, 128), np.uint8)
+    ks = np.ones((P, 64), np.float32)
+    page = 5
+    for j, (vec, s) in enumerate(zip(g["keys"]["vectors_first_two_dims"], g["keys"]["scales"])):
+        kI[page, j, 0] = code[vec[0]] if vec[0] != 0 else 0
+        kI[page, j, 1] = code[vec[1]] if vec[1] != 0 else 0
+        ks[page, j] = s
+    T = len(g["queries"])
+    qI = np.zeros((T, 2, 128), np.uint8)
+    qs = np.zeros(T, np.float32)
+    w = np.zeros((T, 2), np.float32)
+    for t, qq in enumerate(g["queries"]):
+        for r, vec in enumerate(qq["heads_first_two_dims"]):
+            qI[t, r, 0] = code[vec[0]] if vec[0] != 0 else 0
+            qI[t, r, 1] = code[vec[1]] if vec[1] != 0 else 0
+        qs[t] = qq["scale"]
+        w[t] = qq["w"]
+    bt = np.array([[page]], np.int32)
+    seq_lens = np.array([3], np.int32)
+    cu_q = np.array([0, 2], np.int32)
+    expected = np.array([[float(x) for x in row] for row in g["expected_I"]])
+    return dict(seq_lens=seq_lens, cu_q=cu_q, block_table=bt, qI=qI, qI_scale=qs, wI=w,
+                kI_cache=kI, kI_scale=ks), expected
+
+
+def test_index_scores_hand_computed(golden_dir):
+    args, expected = _hand_case(golden_dir)
+    got = O.index_scores(**args)
+    assert got.shape == expected.shape
+    assert np.array_equal(got, expected)
+
+
+def test_query_positions_decode_and_mtp():
+    req, pos = O.query_positions([5, 9, 3], [0, 1, 3, 6])
+    assert list(req) == [0, 1, 1, 2, 2, 2]
+    assert list(pos) == [4, 7, 8, 0, 1, 2]
+
+
+def _small_batch(seq_lens, m, nhI=4, H=8, seed=3, extra_pages=2):
+    wl = synth.custom("tiny", seq_lens, m, n_heads_index=nhI, topk=8, n_heads=H)
+    return synth.make_batch(wl, seed=seed, extra_pages=extra_pages)
+
+
+def _score_args(bt):
+    return dict(seq_lens=bt.seq_lens, cu_q=bt.cu_q, block_table=bt.block_table, qI=bt.qI,
+                qI_scale=bt.qI_scale, wI=bt.wI, kI_cache=bt.kI_cache, kI_scale=bt.kI_scale)
+
+
+def test_index_scores_head_permutation_invariant():
+    bt = _small_batch([70, 33], [3, 2], nhI=8)
+    base = O.index_scores(**_score_args(bt))
+    perm = np.random.default_rng(0).permutation(8)
+    a = _score_args(bt)
+    a["qI"] = bt.qI[:, perm]
+    a["wI"] = bt.wI[:, perm]
+    got = O.index_scores(**a)
+    fin = np.isfinite(base)
+    assert np.array_equal(np.isfinite(got), fin)
+    np.testing.assert_allclose(got[fin], base[fin], rtol=1e-12, atol=1e-12)
+
+
+def test_index_scores_positive_homogeneity_and_selection():
+    bt = _small_batch([90], [4], nhI=4)
+    a = _score_args(bt)
+    base = O.index_scores(**a)
+    a["qI_scale"] = bt.qI_scale * np.float32(4.0)
+    got = O.index_scores(**a)
+    fin = np.isfinite(base)
+    np.testing.assert_allclose(got[fin], 4.0 * base[fin], rtol=1e-12)
+    _, pos = O.query_positions(bt.seq_lens, bt.cu_q)
+    assert np.array_equal(O.topk(base, pos, 8), O.topk(got, pos, 8))
+
+
+def test_index_scores_single_head_is_textbook_dot():
+    """1 head, w = 1, all products positive: I_tj = (s^q q) . (s^k k_j) exactly."""
+    rng = np.random.default_rng(5)
+    n = 10
+    qf = np.abs(rng.standard_normal((1, 1, 128)).astype(np.float32))
+    kf = np.abs(rng.standard_normal((1, 64, 128)).astype(np.float32))
+    qc, qs = synth.quantize_e4m3_per_token(qf)
+    kc, ksc = synth.quantize_e4m3_per_token(kf.reshape(64, 128))
+    qv = torch.from_numpy(qc.reshape(1, 128)).view(torch.float8_e4m3fn).double().numpy() * qs[0]
+    kv = torch.from_numpy(kc).view(torch.float8_e4m3fn).double().numpy() * ksc[:, None].astype(np.float64)
+    want = np.array([float(np.dot(qv[0], kv[j])) for j in range(n)])
+    got = O.index_scores(seq_lens=np.array([n], np.int32), cu_q=np.array([0, 1], np.int32),
+                         block_table=np.array([[0]], np.int32), qI=qc, qI_scale=qs,
+                         wI=np.ones((1, 1), np.float32), kI_cache=kc.reshape(1, 64, 128),
+                         kI_scale=ksc.reshape(1, 64))
+    np.testing.assert_allclose(got[0], want, rtol=1e-12)
+
+
+def test_index_scores_paging_invariant():
+    """Moving pages around the pool (and the block table with them) changes nothing."""
+    bt = _small_batch([130, 64, 7], [2, 1, 3], nhI=4, extra_pages=3)
+    base = O.index_scores(**_score_args(bt))
+    P = bt.num_pages
+    perm = np.random.default_rng(9).permutation(P)          # new slot of old page i is perm[i]
+    kI2 = np.empty_like(bt.kI_cache)
+    ks2 = np.empty_like(bt.kI_scale)
+    kI2[perm] = bt.kI_cache
+    ks2[perm] = bt.kI_scale
+    table = np.where(bt.block_table >= 0, perm[np.maximum(bt.block_table, 0)], -1).astype(np.int32)
+    a = _score_args(bt)
+    a.update(kI_cache=kI2, kI_scale=ks2, block_table=table)
+    got = O.index_scores(**a)
+    assert np.array_equal(got, base)
+
+
+def test_index_scores_causal_mask():
+    bt = _small_batch([40, 12], [5, 12], nhI=2)
+    sc = O.index_scores(**_score_args(bt))
+    _, pos = O.query_positions(bt.seq_lens, bt.cu_q)
+    for t in range(len(pos)):
+        assert np.all(np.isfinite(sc[t, : pos[t] + 1]))
+        assert np.all(np.isneginf(sc[t, pos[t] + 1:]))
+
+
+# ---------------------------------------------------------------------------------------------
+# TopK
+
+def test_topk_worked_example(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "topk_worked_example_p5.json")))
+    s = np.array(g["scores_1based_positions_1_to_8"])
+    S = O.topk_select(s, g["k"])
+    assert sorted(S.tolist()) == g["expected_S_0based"]
+    assert sorted((S + 1).tolist()) == g["expected_S_1based"]
+
+
+def test_topk_worked_example_through_indexer():
+    """t=8 (1-based), k=3: keys at positions 2, 5, 8 aligned with the query's positive head
+    and all others anti-aligned give S_8 = {2, 5, 8} from the actual scoring function."""
+    code_one, code_mone = 0x38, 0xB8
+    kI = np.zeros((1, 64, 128), np.uint8)
+    for j in range(8):
+        kI[0, j, 0] = code_one if (j + 1) in (2, 5, 8) else code_mone
+    ks = np.ones((1, 64), np.float32)
+    ks[0, 1], ks[0, 4], ks[0, 7] = 3.0, 2.0, 1.0
+    qI = np.zeros((1, 1, 128), np.uint8)
+    qI[0, 0, 0] = code_one
+    sc = O.index_scores(seq_lens=np.array([8], np.int32), cu_q=np.array([0, 1], np.int32),
+                        block_table=np.array([[0]], np.int32), qI=qI, qI_scale=np.ones(1, np.float32),
+                        wI=np.ones((1, 1), np.float32), kI_cache=kI, kI_scale=ks)
+    S = O.topk_select(sc[0], 3)
+    assert sorted((S + 1).tolist()) == [2, 5, 8]
+
+
+def test_topk_matches_argpartition():
+    rng = np.random.default_rng(11)
+    for L, k in [(100, 7), (5000, 2048), (4096, 2048), (3000, 1)]:
+        s = rng.standard_normal(L)
+        S = O.topk_select(s, k)
+        want = set(np.argpartition(-s, k - 1)[:k].tolist())
+        assert set(S.tolist()) == want
+
+
+def test_topk_dense_fallback_and_padding():
+    s = np.array([0.3, -1.0, 2.0])
+    S = O.topk_select(s, 5)
+    assert sorted(S[:3].tolist()) == [0, 1, 2]
+    assert S[3:].tolist() == [-1, -1]
+
+
+def test_topk_ties_smaller_position_first():
+    s = np.array([1.0, 5.0, 1.0, 1.0, 5.0, 1.0])
+    assert O.topk_select(s, 3).tolist() == [1, 4, 0]
+
+
+def test_needles_are_selected():
+    wl = synth.custom("needles", [4096] * 2, [1, 2], n_heads_index=16, topk=256, n_heads=4,
+                      needles="decode", n_needles=6)
+    bt = synth.make_batch(wl, seed=0)
+    req, pos = O.query_positions(bt.seq_lens, bt.cu_q)
+    for t, j in bt.needles:
+        I = O.index_scores_row(t, req, pos, bt.block_table, bt.qI, bt.qI_scale, bt.wI,
+                               bt.kI_cache, bt.kI_scale)
+        assert j in set(O.topk_select(I, 256).tolist())
+
+
+# ---------------------------------------------------------------------------------------------
+# sparse attention
+
+def _sdpa(q, k, v, mask, scale):
+    return torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v), attn_mask=torch.from_numpy(mask),
+        scale=scale).numpy()
+
+
+def _mla_batch(L, H=4, seed=2):
+    wl = synth.custom("mla", [L], [L], n_heads_index=2, topk=L, n_heads=H)
+    return synth.make_batch(wl, seed=seed, extra_pages=1)
+
+
+def _latent_rows(bt, b, n):
+    pages, slots = O.physical_rows(bt.block_table[b], np.arange(n))
+    return torch.from_numpy(bt.kv_cache[pages, slots].view(np.int16)).view(torch.bfloat16).double().numpy()
+
+
+def test_sparse_mla_dense_when_k_covers_prefix():
+    """With k >= p+1 the sparse output equals dense causal softmax attention (torch SDPA)."""
+    L, H = 70, 4
+    bt = _mla_batch(L, H)
+    tau = O.default_softmax_scale()
+    _, pos = O.query_positions(bt.seq_lens, bt.cu_q)
+    S = np.full((L, L), -1, np.int32)
+    for t in range(L):
+        S[t, : t + 1] = np.arange(t + 1)[::-1]
+    out, lse = O.sparse_mla(bt.seq_lens, bt.cu_q, bt.block_table, bt.q, bt.kv_cache, S, tau)
+    c = _latent_rows(bt, 0, L)                                           # [L, 576]
+    q = torch.from_numpy(bt.q.view(np.int16)).view(torch.bfloat16).double().numpy()   # [L, H, 576]
+    qh = np.ascontiguousarray(q.transpose(1, 0, 2))                      # [H, L, 576]
+    causal = np.where(np.tril(np.ones((L, L), bool)), 0.0, -np.inf)
+    ref = _sdpa(qh, np.broadcast_to(c, (H, L, 576)).copy(),
+                np.broadcast_to(c[:, :512], (H, L, 512)).copy(), causal, tau)
+    np.testing.assert_allclose(out, ref.transpose(1, 0, 2), rtol=1e-10, atol=1e-12)
+    logits = tau * np.einsum("thd,jd->thj", q, c) + causal[:, None, :]
+    ref_lse = torch.logsumexp(torch.from_numpy(logits), dim=-1).numpy()
+    np.testing.assert_allclose(lse, ref_lse, rtol=1e-12, atol=1e-12)
+
+
+def test_sparse_mla_equals_masked_dense_form():
+    """Gathering S_t equals softmax(QK^T/sqrt(d) + M) V with M = 0 on S_t, -inf elsewhere."""
+    L, H = 90, 3
+    bt = _mla_batch(L, H, seed=4)
+    tau = O.default_softmax_scale()
+    rng = np.random.default_rng(7)
+    k = 11
+    S = np.full((L, k), -1, np.int32)
+    mask = np.full((L, L), -np.inf)
+    for t in range(L):
+        sel = rng.choice(t + 1, size=min(k, t + 1), replace=False)
+        S[t, : sel.size] = sel
+        mask[t, sel] = 0.0
+    out, _ = O.sparse_mla(bt.seq_lens, bt.cu_q, bt.block_table, bt.q, bt.kv_cache, S, tau)
+    c = _latent_rows(bt, 0, L)
+    q = torch.from_numpy(bt.q.view(np.int16)).view(torch.bfloat16).double().numpy()
+    ref = _sdpa(np.ascontiguousarray(q.transpose(1, 0, 2)), np.broadcast_to(c, (H, L, 576)).copy(),
+                np.broadcast_to(c[:, :512], (H, L, 512)).copy(), mask, tau)
+    np.testing.assert_allclose(out, ref.transpose(1, 0, 2), rtol=1e-10, atol=1e-12)
+
+
+def test_sparse_mla_single_index_returns_value_row():
+    L = 20
+    bt = _mla_batch(L, 2, seed=6)
+    S = np.full((L, 4), -1, np.int32)
+    S[:, 0] = 3
+    out, _ = O.sparse_mla(bt.seq_lens, bt.cu_q, bt.block_table, bt.q, bt.kv_cache, S, 0.1)
+    c = _latent_rows(bt, 0, L)
+    for t in range(L):
+        assert np.array_equal(out[t], np.broadcast_to(c[3, :512], out[t].shape))
+
+
+def test_sparse_mla_shift_invariant_and_order_free():
+    L = 40
+    bt = _mla_batch(L, 2, seed=8)
+    rng = np.random.default_rng(1)
+    S = np.stack([rng.permutation(L)[:16] for _ in range(L)]).astype(np.int32)
+    o1, l1 = O.sparse_mla(bt.seq_lens, bt.cu_q, bt.block_table, bt.q, bt.kv_cache, S, 0.07)
+    o2, l2 = O.sparse_mla(bt.seq_lens, bt.cu_q, bt.block_table, bt.q, bt.kv_cache, S[:, ::-1].copy(), 0.07)
+    np.testing.assert_allclose(o1, o2, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(l1, l2, rtol=1e-12)
+
+
+def test_softmax_scale_reading():
+    assert O.default_softmax_scale() == 1.0 / math.sqrt(192.0)
+
+
+# ---------------------------------------------------------------------------------------------
+# cost model against the page's printed table
+
+def test_cost_model_matches_printed_table(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "cost_table_p1.json")))
+    assert round(CM.pair_flops_mla_absorbed() / 1e3) == g["pair_flops_mla_k"]
+    assert round(CM.pair_flops_indexer() / 1e3) == g["pair_flops_indexer_k"]
+    assert round(100 * CM.bytes_per_token_index() / CM.bytes_per_token_latent()) == g["index_cache_overhead_pct"]
+    for row in g["rows"]:
+        dec, rd, pre = CM.per_layer_costs(row["L"])
+        assert [round(x / 1e9, 2) for x in dec] == row["decode_gflops"]
+        assert round(dec[0] / dec[1], 1) == row["decode_ratio"]
+        assert [round(x / 2 ** 20, 1) for x in rd] == row["read_mib"]
+        assert round(rd[0] / rd[1], 1) == row["read_ratio"]
+        assert [round(x / 1e12, 1) for x in pre] == row["prefill_tflops"]
+        assert round(pre[0] / pre[1], 1) == row["prefill_ratio"]
