@@ -1,0 +1,401 @@
+"""Benchmark of the DSA hot path (indexer + top-k + sparse MLA) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one `dsa_layer` call (plan, Lightning-Indexer scores, top-k, sparse MLA) over one batch
+of the workload, inputs resident in HBM. Each timed step is bracketed by CUDA events on the
+launching stream, with a 256 MiB L2 flush (untimed) between steps. Under torchrun every rank runs
+its own batch (weak scaling, no collective on the data path); rank 0 prints one JSON line with the
+max-over-ranks time.
+
+The JSON line also carries
+  roofline      the dominant kernel's achieved algorithmic bytes/s against the measured HBM peak,
+                from per-stage CUDA-event timings of the same kernels;
+  e2e           the same metric through the public API with host (pinned) inputs: per step the
+                queries and batch metadata go host->device and the output comes back; the paged
+                caches stay resident (they are the cache, not per-step inputs);
+  cpu_baseline  the CPU oracle (float64 numpy) timed on this host on a bounded sample of rows.
+`--impl reference` times that oracle alone as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "DSA layer µs (indexer+top-k+sparse MLA), query tok/s; % of HBM/FP8 roofline"
+UNIT = "query tok/s"
+DEFAULT_WORKLOAD = "decode_64x16k"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# ---------------------------------------------------------------------------------------------
+# algorithmic work per step (what the method must move / compute), from the workload's sizes
+
+def algorithmic(hb):
+    """Bytes each kernel must move and FLOPs it must do for one step of this batch."""
+    req, pos = _positions(hb)
+    T = hb.total_q
+    nhI = hb.qI.shape[1]
+    H = hb.q.shape[1]
+    k = hb.wl.topk
+    vis = pos + 1                                   # visible positions per query row
+    sel = np.minimum(vis, k)                        # selected positions per row
+    # indexer: every request's visible keys once per query group (decode: once per request), the
+    # queries, weights and scales, and the score rows written
+    keys_per_req = np.zeros(len(hb.seq_lens), np.int64)
+    for b in range(len(hb.seq_lens)):
+        m = int(hb.cu_q[b + 1] - hb.cu_q[b])
+        if m:
+            keys_per_req[b] = int(hb.seq_lens[b])
+    idx_bytes = int(keys_per_req.sum()) * (128 + 4) + T * (nhI * 128 + 4 + nhI * 4) + int(vis.sum()) * 4
+    idx_flops = int(vis.sum()) * 2 * nhI * 128
+    topk_bytes = int(vis.sum()) * 4 + T * k * 4
+    mla_bytes = int(sel.sum()) * (576 * 2 + 4) + T * H * 576 * 2 + T * H * 512 * 2
+    mla_flops = int(sel.sum()) * (2 * H * 576 + 2 * H * 512)
+    return dict(index_scores=(idx_bytes, idx_flops), topk=(topk_bytes, 0), sparse_mla=(mla_bytes, mla_flops))
+
+
+def _positions(hb):
+    req, pos = hb.row_positions()
+    return req, pos
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        loaded = [x for x in sm if mx is None or x >= 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------------
+# oracle timing (CPU baseline / reference arm)
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n and n[0]:
+            return int(n[0])
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def time_oracle(hb, budget_s: float = 12.0, max_rows: int = 64):
+    """Run the oracle on a bounded sample of query rows; returns (rows/s, rows, seconds)."""
+    from oracle import dsa_oracle as O
+    req, pos = O.query_positions(hb.seq_lens, hb.cu_q)
+    T = hb.total_q
+    tau = hb.wl.softmax_scale
+    k = hb.wl.topk
+    order = np.random.default_rng(0).permutation(T)
+    done, t0 = 0, time.perf_counter()
+    for t in order[:max_rows]:
+        I = O.index_scores_row(int(t), req, pos, hb.block_table, hb.qI, hb.qI_scale, hb.wI, hb.kI_cache,
+                               hb.kI_scale)
+        S = O.topk_select(I, k)
+        O.sparse_mla_row(int(t), req, S, hb.block_table, hb.q, hb.kv_cache, tau)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return done / dt, done, dt
+
+
+# ---------------------------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    from sparse_attention_12_b200 import synth
+    wl = synth.workload(args.workload)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        hb = synth.make_batch(wl, seed=0)
+        budget = max(2.0, min(60.0, 8.0 * max(args.steps, 1) / max(args.steps + args.warmup, 1)))
+        for _ in range(args.warmup):
+            time_oracle(hb, budget_s=0.5, max_rows=1)
+        per_step = []
+        rows_total, secs_total = 0, 0.0
+        for _ in range(args.steps):
+            rate, rows, dt = time_oracle(hb, budget_s=budget / max(args.steps, 1), max_rows=hb.total_q)
+            per_step.append(hb.total_q / rate)   # seconds a full step would take at this rate
+            rows_total += rows
+            secs_total += dt
+        value = rows_total / secs_total
+        ms = 1e3 * hb.total_q / value
+        cores = blas_threads()
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": wl.name, "requests": wl.batch, "query_rows": wl.total_q,
+                           "context": max(wl.seq_lens), "topk": wl.topk, "index_heads": wl.n_heads_index,
+                           "heads": wl.n_heads},
+                "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                 "sample": f"{rows_total} query rows of {wl.name}, full path per row, "
+                                           f"extrapolated to the {hb.total_q}-row step"},
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import torch
+    import sparse_attention_12_b200 as dsa
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local_rank if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    dsa.load()
+
+    hb = synth.make_batch(wl, seed=rank)
+    db = dsa.DeviceBatch(hb, device=dev)
+    T = hb.total_q
+    stream = torch.cuda.current_stream()
+    out = torch.empty((T, db.H, 512), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(16, dsa.layer_workspace_size(db.batch, db.nhI, db.H, db.k)), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        dsa.layer(db.batch, db.qI, db.qI_scale, db.wI, db.kI_cache, db.kI_scale, db.q, db.kv_cache, db.k,
+                  db.softmax_scale, out=out, ws=ws)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    plan_ws = ws  # the plan lives at the start of the layer workspace
+    status = dsa.status_read(plan_ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    barrier()
+    with sampler:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        barrier()
+    times = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = statistics.mean(times)
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms = float(ms_t.item())
+    value = world * T / (ms / 1e3)
+
+    # per-stage timings of the same kernels (roofline of the dominant one)
+    plan_t = dsa.plan(db.batch, db.nhI)
+    ld = (hb.max_seq_len + 127) // 128 * 128
+    scores = torch.empty((T, ld), dtype=torch.float32, device=dev)
+    S = torch.empty((T, db.k), dtype=torch.int32, device=dev)
+    mla_ws_n = dsa.load().dsa_sparse_mla_workspace_size(db.batch.ref(), db.H, db.k)
+    mla_ws = torch.empty(max(16, mla_ws_n), dtype=torch.uint8, device=dev)
+    stages = {
+        "index_scores": lambda: dsa.index_scores(db.batch, plan_t, db.qI, db.qI_scale, db.wI, db.kI_cache,
+                                                 db.kI_scale, scores=scores, ld=ld),
+        "topk": lambda: dsa.topk(db.batch, plan_t, scores, db.k, S=S),
+        "sparse_mla": lambda: dsa.sparse_mla(db.batch, plan_t, db.q, db.kv_cache, S, db.softmax_scale, out=out,
+                                             ws=mla_ws),
+    }
+    for fn in stages.values():
+        fn()
+    stage_ms = {n: [] for n in stages}
+    for i in range(max(3, min(args.steps, 20))):
+        for name, fn in stages.items():
+            flush.fill_(i & 0xFF)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            stage_ms[name].append(a.elapsed_time(b))
+    stage_ms = {n: statistics.mean(v) for n, v in stage_ms.items()}
+    work = algorithmic(hb)
+    hbm_peak, tf_peak, peak_src = measured_peaks()
+    dominant = max(stage_ms, key=stage_ms.get)
+    dom_bytes = work[dominant][0]
+    achieved = dom_bytes / (stage_ms[dominant] / 1e3) / 1e9
+    stage_report = {n: {"us": 1e3 * stage_ms[n], "GBps": work[n][0] / (stage_ms[n] / 1e3) / 1e9,
+                        "TFLOPs": work[n][1] / (stage_ms[n] / 1e3) / 1e12 if work[n][1] else 0.0}
+                    for n in stages}
+    total_bytes = sum(w[0] for w in work.values())
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda t: t.cpu().pin_memory()
+        h_in = {"qI": pin(db.qI.view(torch.uint8)), "qI_scale": pin(db.qI_scale), "wI": pin(db.wI),
+                "q": pin(db.q), "seq_lens": pin(db.batch.seq_lens), "cu_q": pin(db.batch.cu_q),
+                "block_table": pin(db.batch.block_table)}
+        d_in = {n: torch.empty_like(t, device=dev) for n, t in h_in.items()}
+        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+        d2h = h_out.numel() * h_out.element_size()
+        batch2 = dsa.Batch(d_in["seq_lens"], d_in["cu_q"], d_in["block_table"], hb.num_pages, T, db.batch.c.max_q,
+                           hb.max_seq_len)
+        qI_d = d_in["qI"].view(torch.float8_e4m3fn)
+
+        def e2e_step():
+            for n in h_in:
+                d_in[n].copy_(h_in[n], non_blocking=True)
+            dsa.layer(batch2, qI_d, d_in["qI_scale"], d_in["wI"], db.kI_cache, db.kI_scale, d_in["q"],
+                      db.kv_cache, db.k, db.softmax_scale, out=out, ws=ws)
+            h_out.copy_(out, non_blocking=True)
+
+        for _ in range(max(args.warmup, 1)):
+            e2e_step()
+        barrier()
+        es, ee = [], []
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            e2e_step()
+            b.record(stream)
+            es.append(a)
+            ee.append(b)
+        barrier()
+        e_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(es, ee))
+        e_t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+        if dist is not None:
+            dist.all_reduce(e_t, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * T / (float(e_t.item()) / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": float(e_t.item())}
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        rate, rows, dt = time_oracle(hb, budget_s=12.0)
+        cpu = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{rows} of the {T} query rows of {wl.name} through the whole path in "
+                         f"{dt:.1f} s (float64 numpy, BLAS threads)"}
+
+    launches_per_step = 4 + (1 if dsa.load().dsa_sparse_mla_workspace_size(db.batch.ref(), db.H, db.k) > 0 else 0)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "layer_us": 1e3 * ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3+bf16 (fp32 accumulate)", "data": "synthetic",
+        "config": {"workload": wl.name, "requests": wl.batch, "query_rows": T, "context": max(wl.seq_lens),
+                   "topk": wl.topk, "index_heads": wl.n_heads_index, "heads": wl.n_heads, "page_size": 64,
+                   "l2": "256 MiB flush between timed steps", "parallelism": f"{world} independent ranks"},
+        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": None, "peak_source": peak_src},
+        "layer_roofline": {"algorithmic_bytes": total_bytes,
+                           "achieved_GBps": total_bytes / (ms / 1e3) / 1e9,
+                           "frac": total_bytes / (ms / 1e3) / 1e9 / hbm_peak},
+        "stages": stage_report,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": sampler.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,139 @@
+/*
+ * dsa.h — C ABI of the B200 (sm_100a) DeepSeek Sparse Attention hot path.
+ *
+ * The path has three steps, each defined on the pages this library follows:
+ *
+ *   1. Lightning-Indexer scores. "DeepSeek Sparse Attention：从 SWA 到稀疏 Attention 计算", section
+ *      "Lightning Indexer：为历史位置打分并选出 top-k", formula for I_tj:
+ *          I_tj = sum_r w_tr * ReLU(q_tr . k_j)   for every visible position j <= t,
+ *      with one shared key k_j per position. The page "MTP 与稀疏注意力：NSA 与 DSA", section
+ *      "稀疏注意力：NSA 与 DSA", fixes 64 heads of width 128 computed in FP8 and a key cache of
+ *      128 FP8 bytes plus a 4-byte scale per token. Here q_tr = s^q_t * e4m3(qI[t][r]) and
+ *      k_j = s^k_j * e4m3(kI[j]) (per-token fp32 scales).
+ *   2. TopK. Same section: S_t = TopK_{j<=t}(I_tj, k); k = 2048 on the pages; when the prefix holds
+ *      no more than k positions every position is taken (the handbook's k = min(L, TOPK)).
+ *   3. Sparse MLA. Same page, section "Sparse Attention：在选中位置上计算 Attention": attention on the
+ *      rows in S_t only, equivalent to softmax(QK^T/sqrt(d_h) + M) V with M = 0 on S_t and -inf
+ *      elsewhere; S_t is shared by all heads. The handbook computes it in the absorbed MLA form:
+ *      a 576-wide bf16 latent row c_j per position (512 + 64 rope) shared by all 128 heads, with
+ *      V = c_j[0:512].
+ *
+ * Conventions for every entry point:
+ *   - Positions are 0-based. Request b has n_b cached positions (its own query tokens included)
+ *     and m_b query tokens; query i of request b sits at position p = n_b - m_b + i and sees
+ *     j in [0, p].
+ *   - All data pointers are DEVICE pointers owned by the caller; the library allocates no memory
+ *     and keeps no global state (thread-safe). Workspace is caller-provided, sized by the
+ *     *_workspace_size functions.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ *     default stream). Nothing synchronises the host.
+ *   - Arguments are checked on the host before anything is launched; a bad argument returns
+ *     DSA_ERR_INVALID_ARG (or DSA_ERR_UNSUPPORTED for a valid but unsupported size) and launches
+ *     nothing. A failed launch returns DSA_ERR_CUDA. Errors found by a kernel at run time (a wait
+ *     that gave up, an index out of range) are recorded in the status word of the plan and read
+ *     back with dsa_status_read.
+ *   - Tensors are dense and row-major in the shapes given; the paged caches use pages of
+ *     DSA_PAGE_SIZE positions; page ids come from block_table.
+ *   - Pointers must be 16-byte aligned.
+ */
+#ifndef DSA_B200_H_
+#define DSA_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DSA_ABI_VERSION 1
+#define DSA_PAGE_SIZE 64   /* positions per cache page */
+#define DSA_D_INDEX 128    /* indexer head width d_h^I */
+#define DSA_D_LATENT 576   /* latent width: 512 + 64 rope */
+#define DSA_D_V 512        /* value width: first 512 latent dims */
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer, small workspace */
+  DSA_ERR_UNSUPPORTED = 2,  /* a size outside what the kernels are built for */
+  DSA_ERR_WORKSPACE = 3,    /* workspace smaller than *_workspace_size */
+  DSA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+  DSA_ERR_TIMEOUT = 5,      /* a kernel wait gave up (read back by dsa_status_read) */
+  DSA_ERR_DEVICE_INDEX = 6  /* a kernel met an index outside its buffers (dsa_status_read) */
+} dsa_status_t;
+
+/* A ragged batch of requests. Shared by every call. */
+typedef struct dsa_batch {
+  int32_t num_requests;      /* B >= 0 */
+  int32_t total_q;           /* T = sum_b m_b, host copy of cu_q[B] */
+  int32_t max_q;             /* max_b m_b (host), >= 1 when T > 0 */
+  int32_t max_seq_len;       /* max_b n_b (host) */
+  int32_t max_pages;         /* columns of block_table, >= ceil(max_seq_len / 64) */
+  int32_t num_pages;         /* pages in the pool: rows of both paged caches */
+  const int32_t* seq_lens;   /* device int32 [B]: n_b, 1 <= n_b <= max_seq_len, n_b >= m_b */
+  const int32_t* cu_q;       /* device int32 [B+1]: query-row offsets, cu_q[0] = 0 */
+  const int32_t* block_table;/* device int32 [B, max_pages]: physical page of logical page i */
+} dsa_batch_t;
+
+/* ---- batch plan --------------------------------------------------------------------------
+ * Per-batch metadata shared by the steps (row -> request/position, indexer work list, status
+ * word). Compute it once per batch; it stays valid while seq_lens/cu_q do not change.
+ * nhI: indexer heads the plan is made for (16, 32, 64 or 128). */
+size_t dsa_plan_workspace_size(const dsa_batch_t* batch, int nhI);
+dsa_status_t dsa_plan(const dsa_batch_t* batch, int nhI, void* plan, size_t plan_bytes, void* stream);
+
+/* Synchronises `stream`, then returns the status word the kernels of the last calls that used
+ * `plan` recorded (DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE_INDEX) and clears it. */
+dsa_status_t dsa_status_read(void* plan, void* stream);
+
+/* ---- step 1: indexer scores -------------------------------------------------------------
+ * qI       e4m3 [T, nhI, 128]   indexer queries (FP8 codes)
+ * qI_scale f32  [T]             s^q_t
+ * wI       f32  [T, nhI]        head weights w_t
+ * kI_cache e4m3 [P, 64, 128]    indexer keys, paged (FP8 codes)
+ * kI_scale f32  [P, 64]         s^k per cached position
+ * scores   f32  [T, ld]         out: I_tj for j <= p; -inf for p < j < min(ld, 128*ceil((p+1)/128));
+ *                               other entries untouched. ld >= max_seq_len, ld % 4 == 0.
+ * Runs as an FP8 tcgen05 GEMM (keys x query-heads) with ReLU, w and the head sum in the epilogue. */
+dsa_status_t dsa_index_scores(const dsa_batch_t* batch, const void* plan, const uint8_t* qI,
+                              const float* qI_scale, const float* wI, int nhI, const uint8_t* kI_cache,
+                              const float* kI_scale, float* scores, int64_t ld, void* stream);
+
+/* ---- step 2: top-k ----------------------------------------------------------------------
+ * scores f32 [T, ld] as written by dsa_index_scores (row t read at j <= p only).
+ * S      int32 [T, k] out: the min(k, p+1) positions with the largest scores, followed by -1.
+ *        Among equal scores the smaller position wins. Selected positions are listed in
+ *        increasing position order. 1 <= k <= 4096. */
+dsa_status_t dsa_topk(const dsa_batch_t* batch, const void* plan, const float* scores, int64_t ld, int k,
+                      int32_t* S, void* stream);
+
+/* ---- step 3: sparse MLA -----------------------------------------------------------------
+ * q        bf16 [T, H, 576]     absorbed MLA queries, 1 <= H <= 128
+ * kv_cache bf16 [P, 64, 576]    latent rows, paged
+ * S        int32 [T, k]         positions per query row (as dsa_topk writes them: the first
+ *                               min(k, p+1) entries are read, negative entries are skipped)
+ * out      bf16 [T, H, 512]     softmax(scale * q . c_j) weighted sum of c_j[0:512] over S_t
+ * lse      f32  [T, H] or NULL  natural-log sum of exp(scale * q . c_j) over S_t (-inf if empty)
+ * ws/ws_bytes: workspace of dsa_sparse_mla_workspace_size bytes (split partial results). */
+size_t dsa_sparse_mla_workspace_size(const dsa_batch_t* batch, int H, int k);
+dsa_status_t dsa_sparse_mla(const dsa_batch_t* batch, const void* plan, const void* q, int H,
+                            const void* kv_cache, const int32_t* S, int k, float softmax_scale, void* out,
+                            float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- the whole path ---------------------------------------------------------------------
+ * Plan, indexer, top-k and sparse MLA in one call (four to five kernel launches, no host
+ * synchronisation). S_out (int32 [T, k]) receives the index sets when not NULL. The plan lives in
+ * `ws`; dsa_status_read takes `ws` as the plan. */
+size_t dsa_layer_workspace_size(const dsa_batch_t* batch, int nhI, int H, int k);
+dsa_status_t dsa_layer(const dsa_batch_t* batch, const uint8_t* qI, const float* qI_scale, const float* wI,
+                       int nhI, const uint8_t* kI_cache, const float* kI_scale, const void* q, int H,
+                       const void* kv_cache, int k, float softmax_scale, void* out, float* lse, int32_t* S_out,
+                       void* ws, size_t ws_bytes, void* stream);
+
+const char* dsa_status_string(dsa_status_t status);
+int dsa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DSA_B200_H_ */

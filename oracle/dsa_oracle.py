@@ -56,6 +56,17 @@ def e4m3_decode(codes) -> np.ndarray:
     return np.where((e == 15) & ((c & 0x7) == 7), np.nan, v)
 
 
+_E4M3_TABLE = None
+
+
+def e4m3_lookup(codes) -> np.ndarray:
+    """e4m3_decode through a 256-entry table built by e4m3_decode itself (same values, faster)."""
+    global _E4M3_TABLE
+    if _E4M3_TABLE is None:
+        _E4M3_TABLE = e4m3_decode(np.arange(256, dtype=np.uint8))
+    return _E4M3_TABLE[np.asarray(codes).astype(np.uint8)]
+
+
 def bf16_decode(bits) -> np.ndarray:
     """Decode bf16 bit patterns (the upper half of an IEEE float32) to float64."""
     b = np.asarray(bits).astype(np.uint16).astype(np.uint32) << np.uint32(16)
@@ -97,8 +108,8 @@ def index_scores_row(t, req, pos, block_table, qI, qI_scale, wI, kI_cache, kI_sc
     """
     b, p = int(req[t]), int(pos[t])
     pages, slots = physical_rows(block_table[b], np.arange(p + 1))
-    k = e4m3_decode(kI_cache[pages, slots]) * np.asarray(kI_scale, np.float64)[pages, slots][:, None]
-    qt = e4m3_decode(qI[t]) * float(qI_scale[t])            # [nhI, 128]
+    k = e4m3_lookup(kI_cache[pages, slots]) * np.asarray(kI_scale, np.float64)[pages, slots][:, None]
+    qt = e4m3_lookup(qI[t]) * float(qI_scale[t])            # [nhI, 128]
     logits = qt @ k.T                                        # [nhI, p+1]: q_tr . k_j
     return np.asarray(wI[t], np.float64) @ np.maximum(logits, 0.0)
 

@@ -1,0 +1,432 @@
+// Lightning-Indexer scores on sm_100a.
+//
+//   I_tj = s^q_t * s^k_j * sum_r w_tr * ReLU(q_tr . k_j),   j <= p_t
+//
+// ("DeepSeek Sparse Attention：从 SWA 到稀疏 Attention 计算", section "Lightning Indexer", formula
+// for I_tj; FP8 with 64 heads of width 128 per "MTP 与稀疏注意力：NSA 与 DSA", section "稀疏注意力：
+// NSA 与 DSA", which names this kernel an FP8 small GEMM + ReLU + weighted sum.) The per-token
+// scales are positive, so they factor out of the ReLU and are applied once per score.
+//
+// GEMM view: M = 128 keys (two 64-position pages of the paged key cache), N = queries x heads of one
+// "group" (<= 256 columns), K = 128 FP8 bytes. One tcgen05 kind::f8f6f4 MMA chain of 4 x K32 per
+// tile accumulates fp32 in TMEM: TMEM lane i holds key i, column q*nhI + r holds head r of query q.
+// The epilogue thread that owns lane i reads its row, applies ReLU, w and the head sum in
+// registers and writes one fp32 score per query; the per-head products never leave the SM.
+//
+// Persistent CTAs (one per SM) walk a contiguous slice of the plan's tile list. Warp roles:
+//   warp 0      TMA producer: key pages (via the block table) into a 6-stage ring, query tiles and
+//               the group's w / s^q into a 2-deep buffer
+//   warp 1      TMEM allocator and single-thread MMA issuer
+//   warps 2..9  epilogue (two warps per TMEM lane quadrant, splitting the group's queries)
+// Decode tiles are HBM-bound (16 KB of keys per 128x64x128 MMA chain); prefill tiles are
+// tensor-bound with the 8 epilogue warps keeping pace with the MMA.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+
+#include "dsa_internal.h"
+#include "dsa_ptx.cuh"
+
+namespace dsa {
+namespace {
+
+constexpr int kStages = 6;
+constexpr int kStageBytes = kIdxTileKeys * kDIdx;  // 16 KB
+constexpr int kQBufBytes = kIdxCols * kDIdx;       // 32 KB
+constexpr int kMaxAcc = 8;
+constexpr int kThreads = 320;
+constexpr int kEpiWarps = 8;
+
+struct __align__(16) GroupMeta {
+  int32_t row0, nq, pos0, req;
+};
+
+struct IdxSmem {
+  // byte offsets relative to the 1024-aligned base
+  static constexpr int kStage0 = 0;
+  static constexpr int kQBuf0 = kStage0 + kStages * kStageBytes;  // 96 KB
+  static constexpr int kW = kQBuf0 + 2 * kQBufBytes;              // 160 KB: float [2][256]
+  static constexpr int kSq = kW + 2 * kIdxCols * 4;               // float [2][16]
+  static constexpr int kMeta = kSq + 2 * 16 * 4;                  // GroupMeta [2]
+  static constexpr int kBars = kMeta + 2 * 16;                    // uint64 barriers
+  static constexpr int kNumBars = 2 * kStages + 4 + 2 * kMaxAcc;
+  static constexpr int kTmemSlot = kBars + kNumBars * 8;
+  static constexpr int kTotal = kTmemSlot + 16;
+  static constexpr int kDynamic = kTotal + 1024;  // slack for the manual 1024-byte alignment
+};
+
+struct IdxParams {
+  BatchDev bd;
+  const PlanHeader* hdr;
+  const int32_t* grp_row0;
+  const int32_t* grp_nq;
+  const int32_t* grp_req;
+  const int32_t* grp_pos0;
+  const int32_t* grp_tile0;
+  const float* qI_scale;
+  const float* wI;
+  const float* kI_scale;
+  float* scores;
+  int64_t ld;
+  int ncols;      // TMEM columns per accumulator buffer (power of two >= 32)
+  int nacc;       // accumulator buffers
+  int qbox_rows;  // query rows per TMA box
+  uint32_t* status;
+};
+
+// Last group g with tile0[g] <= u.
+__device__ __forceinline__ int find_group(const int32_t* tile0, int G, int u) {
+  int lo = 0, hi = G;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(tile0 + mid) <= u)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
+
+template <int NHI>
+__global__ void __launch_bounds__(kThreads, 1)
+    index_scores_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                        const IdxParams p) {
+  constexpr int QPG = kIdxCols / NHI;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  float* g_w = reinterpret_cast<float*>(base + IdxSmem::kW);
+  float* g_sq = reinterpret_cast<float*>(base + IdxSmem::kSq);
+  GroupMeta* g_meta = reinterpret_cast<GroupMeta*>(base + IdxSmem::kMeta);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + IdxSmem::kBars);
+  uint64_t* kfull = bars;
+  uint64_t* kempty = bars + kStages;
+  uint64_t* qfull = bars + 2 * kStages;
+  uint64_t* qempty = qfull + 2;
+  uint64_t* tfull = qempty + 2;
+  uint64_t* tempty = tfull + kMaxAcc;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + IdxSmem::kTmemSlot);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int G = p.hdr->num_groups;
+  const int U = p.hdr->total_tiles;
+  const int u0 = static_cast<int>((static_cast<int64_t>(U) * blockIdx.x) / gridDim.x);
+  const int u1 = static_cast<int>((static_cast<int64_t>(U) * (blockIdx.x + 1)) / gridDim.x);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&kfull[s], 1);
+      mbar_init(&kempty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&qfull[b], 1);
+      mbar_init(&qempty[b], 1 + kEpiWarps);
+    }
+    for (int a = 0; a < kMaxAcc; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], kEpiWarps);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&kmap);
+    tma_prefetch_desc(&qmap);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (u0 < u1) {
+    if (warp == 0) {
+      // ---------------- producer ----------------
+      int g = find_group(p.grp_tile0, G, u0);
+      int gstart = __ldg(p.grp_tile0 + g), gend = __ldg(p.grp_tile0 + g + 1);
+      GroupMeta gm{};
+      int qcount = 0;
+      int pg_base = -1;  // first logical page held in `pg_cache`
+      int pg_cache = 0;
+      bool ok = true;
+      for (int u = u0, it = 0; u < u1 && ok; ++u, ++it) {
+        const bool newg = (u == u0) || (u == gend);
+        if (u == gend) {
+          ++g;
+          gstart = gend;
+          gend = __ldg(p.grp_tile0 + g + 1);
+        }
+        if (newg) {
+          const int qb = qcount & 1;
+          if (lane == 0) ok = mbar_wait(&qempty[qb], ((qcount >> 1) & 1) ^ 1, p.status, kDevErrTimeout);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          gm.row0 = __ldg(p.grp_row0 + g);
+          gm.nq = __ldg(p.grp_nq + g);
+          gm.pos0 = __ldg(p.grp_pos0 + g);
+          gm.req = __ldg(p.grp_req + g);
+          for (int idx = lane; idx < QPG * NHI; idx += 32) {
+            const int q = idx / NHI;
+            g_w[qb * kIdxCols + idx] = (q < gm.nq) ? __ldg(p.wI + static_cast<int64_t>(gm.row0 + q) * NHI + (idx % NHI)) : 0.f;
+          }
+          if (lane < QPG) g_sq[qb * 16 + lane] = (lane < gm.nq) ? __ldg(p.qI_scale + gm.row0 + lane) : 0.f;
+          if (lane == 0) g_meta[qb] = gm;
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&qfull[qb], static_cast<uint32_t>(p.qbox_rows * kDIdx));
+            tma_load_2d(base + IdxSmem::kQBuf0 + qb * kQBufBytes, &qmap, 0, gm.row0 * NHI, &qfull[qb]);
+          }
+          ++qcount;
+          pg_base = -1;
+        }
+        const int kt = u - gstart;
+        const int lp0 = 2 * kt;
+        // block-table window of 32 logical pages, refreshed every 16 tiles
+        if (pg_base < 0 || lp0 >= pg_base + 32) {
+          pg_base = lp0;
+          const int lp = pg_base + lane;
+          const int npages = (gm.pos0 + gm.nq - 1) / kPage + 1;
+          pg_cache = (lp < npages) ? __ldg(p.bd.block_table + static_cast<int64_t>(gm.req) * p.bd.max_pages + lp) : 0;
+        }
+        const int pg0 = __shfl_sync(0xffffffffu, pg_cache, lp0 - pg_base);
+        const int pg1 = __shfl_sync(0xffffffffu, pg_cache, lp0 + 1 - pg_base);
+        if (lane == 0) {
+          const int s = it % kStages;
+          ok = mbar_wait(&kempty[s], ((it / kStages) & 1) ^ 1, p.status, kDevErrTimeout);
+          if (ok) {
+            const int p_last = gm.pos0 + gm.nq - 1;
+            const bool v1 = (lp0 + 1) * kPage <= p_last;
+            if (pg0 < 0 || pg0 >= p.bd.num_pages || (v1 && (pg1 < 0 || pg1 >= p.bd.num_pages)))
+              report_error(p.status, kDevErrIndex);
+            uint8_t* dst = base + IdxSmem::kStage0 + s * kStageBytes;
+            mbar_arrive_expect_tx(&kfull[s], static_cast<uint32_t>((v1 ? 2 : 1) * kPage * kDIdx));
+            tma_load_2d(dst, &kmap, 0, pg0 * kPage, &kfull[s]);
+            if (v1) tma_load_2d(dst + kPage * kDIdx, &kmap, 0, pg1 * kPage, &kfull[s]);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+      }
+    } else if (warp == 1) {
+      // ---------------- MMA issuer ----------------
+      if (lane == 0) {
+        int g = find_group(p.grp_tile0, G, u0);
+        int gend = __ldg(p.grp_tile0 + g + 1);
+        int nq = 0, qcount = 0, qb = 0;
+        bool ok = true;
+        for (int u = u0, it = 0; u < u1 && ok; ++u, ++it) {
+          const bool newg = (u == u0) || (u == gend);
+          if (u == gend) {
+            ++g;
+            gend = __ldg(p.grp_tile0 + g + 1);
+          }
+          if (newg) {
+            qb = qcount & 1;
+            ok = mbar_wait(&qfull[qb], (qcount >> 1) & 1, p.status, kDevErrTimeout);
+            if (!ok) break;
+            nq = __ldg(p.grp_nq + g);
+            ++qcount;
+          }
+          const int s = it % kStages;
+          const int a = it % p.nacc;
+          ok = mbar_wait(&kfull[s], (it / kStages) & 1, p.status, kDevErrTimeout) &&
+               mbar_wait(&tempty[a], ((it / p.nacc) & 1) ^ 1, p.status, kDevErrTimeout);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t idesc = umma_idesc(128, static_cast<uint32_t>(nq * NHI), 0, 0, 0);
+          const uint32_t a_addr = smem_u32(base + IdxSmem::kStage0 + s * kStageBytes);
+          const uint32_t b_addr = smem_u32(base + IdxSmem::kQBuf0 + qb * kQBufBytes);
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * p.ncols);
+#pragma unroll
+          for (int k = 0; k < kDIdx / 32; ++k) {
+            mma_f8_ss(d_tmem, umma_desc_sw128(a_addr + 32 * k, 16, 1024), umma_desc_sw128(b_addr + 32 * k, 16, 1024),
+                      idesc, k > 0 ? 1u : 0u);
+          }
+          mma_commit(&kempty[s]);
+          mma_commit(&tfull[a]);
+          if (u + 1 == gend || u + 1 == u1) mma_commit(&qempty[qb]);
+        }
+      }
+      __syncwarp();
+    } else {
+      // ---------------- epilogue ----------------
+      const int ew = warp - 2;
+      const int quad = warp & 3;
+      const int half = ew >> 2;
+      const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+      int g = find_group(p.grp_tile0, G, u0);
+      int gstart = __ldg(p.grp_tile0 + g), gend = __ldg(p.grp_tile0 + g + 1);
+      int qcount = 0, qb = 0;
+      GroupMeta gm{};
+      bool ok = true;
+      for (int u = u0, it = 0; u < u1 && ok; ++u, ++it) {
+        const bool newg = (u == u0) || (u == gend);
+        if (u == gend) {
+          ++g;
+          gstart = gend;
+          gend = __ldg(p.grp_tile0 + g + 1);
+        }
+        if (newg) {
+          qb = qcount & 1;
+          ok = __all_sync(0xffffffffu, mbar_wait(&qfull[qb], (qcount >> 1) & 1, p.status, kDevErrTimeout));
+          if (!ok) break;
+          gm = g_meta[qb];
+          ++qcount;
+        }
+        const int kt = u - gstart;
+        const int j = kt * kIdxTileKeys + quad * 32 + lane;
+        const int p_last = gm.pos0 + gm.nq - 1;
+        float sk = 0.f;
+        if (j <= p_last) {
+          int pg = __ldg(p.bd.block_table + static_cast<int64_t>(gm.req) * p.bd.max_pages + j / kPage);
+          pg = min(max(pg, 0), p.bd.num_pages - 1);
+          sk = __ldg(p.kI_scale + static_cast<int64_t>(pg) * kPage + (j % kPage));
+        }
+        const int a = it % p.nacc;
+        ok = __all_sync(0xffffffffu, mbar_wait(&tfull[a], (it / p.nacc) & 1, p.status, kDevErrTimeout));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t t_row = tmem_base + lane_base + static_cast<uint32_t>(a * p.ncols);
+        for (int q = half; q < gm.nq; q += 2) {
+          const float* w = g_w + qb * kIdxCols + q * NHI;
+          float acc = 0.f;
+          if constexpr (NHI % 32 == 0) {
+#pragma unroll
+            for (int c = 0; c < NHI / 32; ++c) {
+              uint32_t v[32];
+              tmem_ld32(t_row + static_cast<uint32_t>(q * NHI + c * 32), v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) acc = fmaf(w[c * 32 + i], fmaxf(__uint_as_float(v[i]), 0.f), acc);
+            }
+          } else {
+            uint32_t v[16];
+            tmem_ld16(t_row + static_cast<uint32_t>(q * NHI), v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc = fmaf(w[i], fmaxf(__uint_as_float(v[i]), 0.f), acc);
+          }
+          float score = acc * g_sq[qb * 16 + q] * sk;
+          if (j > gm.pos0 + q) score = -INFINITY;
+          if (j < p.ld) p.scores[static_cast<int64_t>(gm.row0 + q) * p.ld + j] = score;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&tempty[a]);
+          if (u + 1 == gend || u + 1 == u1) mbar_arrive(&qempty[qb]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+}  // namespace
+
+int make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* ptr, uint64_t inner,
+                 uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return static_cast<int>(cudaErrorNotSupported);
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  (void)elem_bytes;
+  CUresult r = fn(map, dtype, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : static_cast<int>(cudaErrorInvalidValue);
+}
+
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
+  }
+  return n;
+}
+
+template <int NHI>
+static int launch_index_scores_t(const BatchDev& b, const void* plan, const uint8_t* qI, const float* qI_scale,
+                                 const float* wI, const uint8_t* kI_cache, const float* kI_scale, float* scores,
+                                 int64_t ld, void* stream) {
+  constexpr int QPG = kIdxCols / NHI;
+  PlanView pv = plan_view(const_cast<void*>(plan), b.B, b.T);
+  IdxParams prm{};
+  prm.bd = b;
+  prm.hdr = pv.hdr;
+  prm.grp_row0 = pv.grp_row0;
+  prm.grp_nq = pv.grp_nq;
+  prm.grp_req = pv.grp_req;
+  prm.grp_pos0 = pv.grp_pos0;
+  prm.grp_tile0 = pv.grp_tile0;
+  prm.qI_scale = qI_scale;
+  prm.wI = wI;
+  prm.kI_scale = kI_scale;
+  prm.scores = scores;
+  prm.ld = ld;
+  const int qmax = b.max_q < QPG ? b.max_q : QPG;
+  int ncols = 32;
+  while (ncols < qmax * NHI) ncols <<= 1;
+  prm.ncols = ncols;
+  prm.nacc = (512 / ncols) < kMaxAcc ? (512 / ncols) : kMaxAcc;
+  prm.qbox_rows = qmax * NHI;
+  prm.status = &pv.hdr->status;
+
+  CUtensorMap kmap, qmap;
+  int e = make_tmap_2d(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, kI_cache, kDIdx,
+                       static_cast<uint64_t>(b.num_pages) * kPage, kDIdx, kDIdx, kPage);
+  if (e) return e;
+  e = make_tmap_2d(&qmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, qI, kDIdx, static_cast<uint64_t>(b.T) * NHI, kDIdx,
+                   kDIdx, static_cast<uint32_t>(prm.qbox_rows));
+  if (e) return e;
+  auto kern = index_scores_kernel<NHI>;
+  cudaError_t ce = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, IdxSmem::kDynamic);
+  if (ce != cudaSuccess) return static_cast<int>(ce);
+  kern<<<num_sms(), kThreads, IdxSmem::kDynamic, static_cast<cudaStream_t>(stream)>>>(kmap, qmap, prm);
+  return static_cast<int>(cudaGetLastError());
+}
+
+int launch_index_scores(const BatchDev& b, const void* plan, const uint8_t* qI, const float* qI_scale,
+                        const float* wI, int nhI, const uint8_t* kI_cache, const float* kI_scale, float* scores,
+                        int64_t ld, void* stream) {
+  switch (nhI) {
+    case 16:
+      return launch_index_scores_t<16>(b, plan, qI, qI_scale, wI, kI_cache, kI_scale, scores, ld, stream);
+    case 32:
+      return launch_index_scores_t<32>(b, plan, qI, qI_scale, wI, kI_cache, kI_scale, scores, ld, stream);
+    case 64:
+      return launch_index_scores_t<64>(b, plan, qI, qI_scale, wI, kI_cache, kI_scale, scores, ld, stream);
+    case 128:
+      return launch_index_scores_t<128>(b, plan, qI, qI_scale, wI, kI_cache, kI_scale, scores, ld, stream);
+    default:
+      return static_cast<int>(cudaErrorInvalidValue);
+  }
+}
+
+}  // namespace dsa

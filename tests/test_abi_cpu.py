@@ -1,0 +1,121 @@
+"""The C-ABI library without a GPU: it loads, exports every declared entry point, and rejects bad
+arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import sparse_attention_12_b200 as dsa
+from sparse_attention_12_b200 import build as dsa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dsa_build.build()
+    return dsa.load()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(dsa_[a-z_0-9]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 11
+    out = subprocess.run(["nm", "-D", "--defined-only", dsa.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (dsa_\w+)", out))
+    for n in names:
+        assert n in exported, n
+        assert hasattr(lib, n)
+    assert set(dsa.EXPORTS) == set(names)
+
+
+def test_abi_version_and_strings(lib):
+    assert lib.dsa_abi_version() == 1
+    for s in range(7):
+        assert lib.dsa_status_string(s).decode() == dsa.STATUS[s]
+    assert lib.dsa_status_string(99).decode() == "unknown status"
+
+
+FAKE = 1 << 20  # an aligned, never-dereferenced "device" address: validation must fail first
+
+
+def batch(B=2, T=3, max_q=2, max_seq_len=300, max_pages=5, num_pages=10):
+    return dsa.DsaBatchC(B, T, max_q, max_seq_len, max_pages, num_pages, FAKE, FAKE, FAKE)
+
+
+def test_plan_rejects_bad_arguments(lib):
+    b = batch()
+    n = lib.dsa_plan_workspace_size(ctypes.byref(b), 64)
+    assert n > 64
+    assert lib.dsa_plan(None, 64, FAKE, n, None) == 1
+    assert lib.dsa_plan(ctypes.byref(b), 48, FAKE, n, None) == 2
+    assert lib.dsa_plan(ctypes.byref(b), 64, FAKE + 4, n, None) == 1       # misaligned
+    assert lib.dsa_plan(ctypes.byref(b), 64, FAKE, n - 1, None) == 3       # workspace
+    bad = batch(max_pages=4)                                               # 300 positions need 5 pages
+    assert lib.dsa_plan(ctypes.byref(bad), 64, FAKE, n, None) == 1
+    nulls = dsa.DsaBatchC(2, 3, 2, 300, 5, 10, None, FAKE, FAKE)
+    assert lib.dsa_plan(ctypes.byref(nulls), 64, FAKE, n, None) == 1
+
+
+def test_empty_batch_is_a_no_op(lib):
+    b = dsa.DsaBatchC(0, 0, 0, 0, 0, 0, None, None, None)
+    assert lib.dsa_index_scores(ctypes.byref(b), None, None, None, None, 64, None, None, None, 0, None) == 0
+    assert lib.dsa_topk(ctypes.byref(b), None, None, 0, 2048, None, None) == 0
+    assert lib.dsa_sparse_mla(ctypes.byref(b), None, None, 128, None, None, 2048, 0.07, None, None, None, 0,
+                              None) == 0
+    assert lib.dsa_layer(ctypes.byref(b), None, None, None, 64, None, None, None, 128, None, 2048, 0.07, None,
+                         None, None, None, 0, None) == 0
+
+
+def test_index_scores_validation(lib):
+    b = batch()
+    call = lambda **kw: lib.dsa_index_scores(
+        ctypes.byref(b), kw.get("plan", FAKE), kw.get("qI", FAKE), FAKE, FAKE, kw.get("nhI", 64),
+        kw.get("kI", FAKE), FAKE, kw.get("scores", FAKE), kw.get("ld", 384), None)
+    assert call(nhI=20) == 2
+    assert call(qI=None) == 1
+    assert call(kI=FAKE + 8) == 1
+    assert call(ld=256) == 1          # ld < max_seq_len
+    assert call(ld=302) == 1          # ld % 4
+    assert call(scores=None) == 1
+
+
+def test_topk_and_mla_validation(lib):
+    b = batch()
+    assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE, 384, 0, FAKE, None) == 2
+    assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE, 384, 5000, FAKE, None) == 2
+    assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE, 100, 16, FAKE, None) == 1
+    mla = lambda **kw: lib.dsa_sparse_mla(
+        ctypes.byref(b), FAKE, kw.get("q", FAKE), kw.get("H", 128), FAKE, FAKE, kw.get("k", 2048),
+        kw.get("scale", 0.07), FAKE, None, kw.get("ws", FAKE), kw.get("ws_bytes", 1 << 30), None)
+    assert mla(H=0) == 2
+    assert mla(H=129) == 2
+    assert mla(k=0) == 2
+    assert mla(scale=0.0) == 1
+    assert mla(scale=float("nan")) == 1
+    assert mla(q=FAKE + 2) == 1
+    need = lib.dsa_sparse_mla_workspace_size(ctypes.byref(b), 128, 2048)
+    assert need > 0          # 3 rows cannot fill the GPU: split partials need workspace
+    assert mla(ws_bytes=need - 1) == 3
+
+
+def test_layer_workspace_accounting(lib):
+    b = batch()
+    n = lib.dsa_layer_workspace_size(ctypes.byref(b), 64, 128, 2048)
+    plan = lib.dsa_plan_workspace_size(ctypes.byref(b), 64)
+    mla = lib.dsa_sparse_mla_workspace_size(ctypes.byref(b), 128, 2048)
+    scores = 4 * 3 * 384
+    S = 4 * 3 * 2048
+    assert n >= plan + scores + S + mla
+    assert n <= plan + scores + S + mla + 4 * 256
+    args = [ctypes.byref(b), FAKE, FAKE, FAKE, 64, FAKE, FAKE, FAKE, 128, FAKE, 2048, 0.07, FAKE, None, None, FAKE]
+    assert lib.dsa_layer(*args, n - 1, None) == 3
+    assert lib.dsa_layer(*args[:4], 40, *args[5:], n, None) == 2
