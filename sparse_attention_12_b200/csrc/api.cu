@@ -105,7 +105,8 @@ dsa_status_t dsa_index_scores(const dsa_batch_t* batch, const void* plan, const 
   if (!valid_nhI(nhI)) return DSA_ERR_UNSUPPORTED;
   if (batch->total_q == 0) return DSA_OK;
   if (!plan || !qI || !qI_scale || !wI || !kI_cache || !kI_scale || !scores) return DSA_ERR_INVALID_ARG;
-  if (!aligned16(plan) || !aligned16(qI) || !aligned16(kI_cache) || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(plan) || !aligned16(qI) || !aligned16(kI_cache) || !aligned16(kI_scale) || !aligned16(scores))
+    return DSA_ERR_INVALID_ARG;
   if (ld < batch->max_seq_len || ld % 4 != 0) return DSA_ERR_INVALID_ARG;
   if (static_cast<int64_t>(batch->total_q) * nhI > (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
   return from_cuda(launch_index_scores(to_dev(batch), plan, qI, qI_scale, wI, nhI, kI_cache, kI_scale, scores, ld,
@@ -164,8 +165,8 @@ dsa_status_t dsa_layer(const dsa_batch_t* batch, const uint8_t* qI, const float*
   if (H < 1 || H > 128 || k < 1 || k > kMaxTopK) return DSA_ERR_UNSUPPORTED;
   if (batch->total_q == 0) return DSA_OK;
   if (!qI || !qI_scale || !wI || !kI_cache || !kI_scale || !q || !kv_cache || !out || !ws) return DSA_ERR_INVALID_ARG;
-  if (!aligned16(qI) || !aligned16(kI_cache) || !aligned16(q) || !aligned16(kv_cache) || !aligned16(out) ||
-      !aligned16(ws))
+  if (!aligned16(qI) || !aligned16(kI_cache) || !aligned16(kI_scale) || !aligned16(q) || !aligned16(kv_cache) ||
+      !aligned16(out) || !aligned16(ws))
     return DSA_ERR_INVALID_ARG;
   if (!(softmax_scale > 0.f)) return DSA_ERR_INVALID_ARG;
   if (static_cast<int64_t>(batch->total_q) * nhI > (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;

@@ -47,7 +47,8 @@ struct IdxSmem {
   static constexpr int kStage0 = 0;
   static constexpr int kQBuf0 = kStage0 + kStages * kStageBytes;  // 96 KB
   static constexpr int kW = kQBuf0 + 2 * kQBufBytes;              // 160 KB: float [2][256]
-  static constexpr int kSq = kW + 2 * kIdxCols * 4;               // float [2][16]
+  static constexpr int kScale = kW + 2 * kIdxCols * 4;            // float [kStages][128]: s^k of the tile
+  static constexpr int kSq = kScale + kStages * kIdxTileKeys * 4; // float [2][16]
   static constexpr int kMeta = kSq + 2 * 16 * 4;                  // GroupMeta [2]
   static constexpr int kBars = kMeta + 2 * 16;                    // uint64 barriers
   static constexpr int kNumBars = 2 * kStages + 4 + 2 * kMaxAcc;
@@ -97,6 +98,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   float* g_w = reinterpret_cast<float*>(base + IdxSmem::kW);
   float* g_sq = reinterpret_cast<float*>(base + IdxSmem::kSq);
+  float* g_scale = reinterpret_cast<float*>(base + IdxSmem::kScale);
   GroupMeta* g_meta = reinterpret_cast<GroupMeta*>(base + IdxSmem::kMeta);
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + IdxSmem::kBars);
   uint64_t* kfull = bars;
@@ -116,7 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&kfull[s], 1);
-      mbar_init(&kempty[s], 1);
+      mbar_init(&kempty[s], 1 + kEpiWarps);  // MMA done with the keys, epilogue with the scales
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&qfull[b], 1);
@@ -201,9 +203,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (pg0 < 0 || pg0 >= p.bd.num_pages || (v1 && (pg1 < 0 || pg1 >= p.bd.num_pages)))
               report_error(p.status, kDevErrIndex);
             uint8_t* dst = base + IdxSmem::kStage0 + s * kStageBytes;
-            mbar_arrive_expect_tx(&kfull[s], static_cast<uint32_t>((v1 ? 2 : 1) * kPage * kDIdx));
+            float* sdst = g_scale + s * kIdxTileKeys;
+            const int q0 = min(max(pg0, 0), p.bd.num_pages - 1), q1 = min(max(pg1, 0), p.bd.num_pages - 1);
+            mbar_arrive_expect_tx(&kfull[s], static_cast<uint32_t>((v1 ? 2 : 1) * kPage * (kDIdx + 4)));
             tma_load_2d(dst, &kmap, 0, pg0 * kPage, &kfull[s]);
-            if (v1) tma_load_2d(dst + kPage * kDIdx, &kmap, 0, pg1 * kPage, &kfull[s]);
+            bulk_load(sdst, p.kI_scale + static_cast<int64_t>(q0) * kPage, kPage * 4, &kfull[s]);
+            if (v1) {
+              tma_load_2d(dst + kPage * kDIdx, &kmap, 0, pg1 * kPage, &kfull[s]);
+              bulk_load(sdst + kPage, p.kI_scale + static_cast<int64_t>(q1) * kPage, kPage * 4, &kfull[s]);
+            }
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -235,14 +243,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           tc_fence_after();
           const uint32_t idesc = umma_idesc(128, static_cast<uint32_t>(nq * NHI), 0, 0, 0);
-          const uint32_t a_addr = smem_u32(base + IdxSmem::kStage0 + s * kStageBytes);
-          const uint32_t b_addr = smem_u32(base + IdxSmem::kQBuf0 + qb * kQBufBytes);
+          const uint64_t ad = umma_desc_sw128(smem_u32(base + IdxSmem::kStage0 + s * kStageBytes), 16, 1024);
+          const uint64_t bd = umma_desc_sw128(smem_u32(base + IdxSmem::kQBuf0 + qb * kQBufBytes), 16, 1024);
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * p.ncols);
 #pragma unroll
-          for (int k = 0; k < kDIdx / 32; ++k) {
-            mma_f8_ss(d_tmem, umma_desc_sw128(a_addr + 32 * k, 16, 1024), umma_desc_sw128(b_addr + 32 * k, 16, 1024),
-                      idesc, k > 0 ? 1u : 0u);
-          }
+          for (int k = 0; k < kDIdx / 32; ++k)  // K step of 32 bytes = +2 in the start-address field
+            mma_f8_ss(d_tmem, ad + 2 * k, bd + 2 * k, idesc, k > 0 ? 1u : 0u);
           mma_commit(&kempty[s]);
           mma_commit(&tfull[a]);
           if (u + 1 == gend || u + 1 == u1) mma_commit(&qempty[qb]);
@@ -277,15 +283,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kt = u - gstart;
         const int j = kt * kIdxTileKeys + quad * 32 + lane;
         const int p_last = gm.pos0 + gm.nq - 1;
-        float sk = 0.f;
-        if (j <= p_last) {
-          int pg = __ldg(p.bd.block_table + static_cast<int64_t>(gm.req) * p.bd.max_pages + j / kPage);
-          pg = min(max(pg, 0), p.bd.num_pages - 1);
-          sk = __ldg(p.kI_scale + static_cast<int64_t>(pg) * kPage + (j % kPage));
-        }
+        const int s = it % kStages;
         const int a = it % p.nacc;
-        ok = __all_sync(0xffffffffu, mbar_wait(&tfull[a], (it / p.nacc) & 1, p.status, kDevErrTimeout));
+        ok = __all_sync(0xffffffffu, mbar_wait(&kfull[s], (it / kStages) & 1, p.status, kDevErrTimeout) &&
+                                         mbar_wait(&tfull[a], (it / p.nacc) & 1, p.status, kDevErrTimeout));
         if (!ok) break;
+        const float sk = (j <= p_last) ? g_scale[s * kIdxTileKeys + quad * 32 + lane] : 0.f;
         tc_fence_after();
         const uint32_t t_row = tmem_base + lane_base + static_cast<uint32_t>(a * p.ncols);
         for (int q = half; q < gm.nq; q += 2) {
@@ -314,6 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
+          mbar_arrive(&kempty[s]);
           mbar_arrive(&tempty[a]);
           if (u + 1 == gend || u + 1 == u1) mbar_arrive(&qempty[qb]);
         }

@@ -10,15 +10,17 @@
 // One CTA per (query row, half of the 512 value dims, split of S_t); one CTA per SM.
 //   * Q (128 heads x 576, bf16): dims 0..319 sit in TMEM and feed the S = Q C^T MMAs as the A
 //     operand; dims 320..575 sit in shared memory (TMA, 128-byte swizzle).
-//   * Latent rows c_j are gathered 32 at a time through the block table with 16-byte cp.async into
-//     a 4-stage ring laid out in the 128-byte-swizzled UMMA layout (9 blocks of 64 dims).
+//   * Latent rows c_j are gathered 32 at a time through the block table with TMA tile::gather4
+//     (4 rows x 64 dims per copy, 72 copies per tile) into a 4-stage ring; the tensor map's 128-byte
+//     swizzle follows the shared-memory address, so 4-row copies at 512-byte steps build the
+//     canonical K-major UMMA layout (9 blocks of 64 dims, 8-row atoms).
 //   * S tile [128 heads x 32 keys] accumulates in TMEM (double-buffered), the softmax warps turn it
 //     into P (bf16) in TMEM, and O[:, half] (128 x 256 fp32) accumulates in TMEM from P x V with
 //     V read from the same shared-memory stage in its MN-major view.
 //   * Online softmax with lazy rescaling: the reference maximum only moves when a tile's maximum
 //     exceeds it by more than 2^8, so O is rarely touched outside the MMAs.
 // TMEM columns: O 0..255 | S 256..319 (2 x 32) | P 320..351 (2 x 16) | Q 352..511 (160).
-// Warps: 0-1 gather producers, 2 MMA issuer (+ TMEM allocator), 3-6 softmax and epilogue.
+// Warps: 0 gather producer (TMA), 1 MMA issuer (+ TMEM allocator), 2-5 softmax and epilogue.
 //
 // Splits (several CTAs over one S_t) write normalised partial outputs and their log-sum-exp to the
 // workspace; a combine kernel merges them: o = sum_s exp(lse_s - lse) o_s.
@@ -45,8 +47,7 @@ constexpr int kQTmemDims = 320;                      // Q dims held in TMEM
 constexpr int kQSmemBlocks = (kDLat - kQTmemDims) / 64;  // 4 blocks in shared memory
 constexpr int kQBlkBytes = 128 * 128;                // 16 KB
 constexpr int kMaxKeysPerCta = 2048;
-constexpr int kThreads = 224;
-constexpr int kProducerThreads = 64;
+constexpr int kThreads = 192;
 constexpr float kRescaleThreshold = 8.0f;            // log2 units
 
 constexpr uint32_t kColO = 0, kColS = 256, kColP = 320, kColQ = 352;
@@ -83,7 +84,8 @@ struct MlaParams {
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
-    sparse_mla_kernel(const __grid_constant__ CUtensorMap qmap, const MlaParams p) {
+    sparse_mla_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kvmap,
+                      const MlaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   int32_t* rows = reinterpret_cast<int32_t*>(base + MlaSmem::kRows);
@@ -110,7 +112,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&kv_full[s], kProducerThreads);
+      mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -123,7 +125,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_full, 1);
     fence_barrier_init();
   }
-  if (warp == 2) {
+  if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -154,6 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (threadIdx.x == 0 && ntiles > 0) {
     tma_prefetch_desc(&qmap);
+    tma_prefetch_desc(&kvmap);
     mbar_arrive_expect_tx(q_full, kQSmemBlocks * kQBlkBytes);
     for (int i = 0; i < kQSmemBlocks; ++i)
       tma_load_2d(base + MlaSmem::kQ + i * kQBlkBytes, &qmap, kQTmemDims + 64 * i, t * H, q_full);
@@ -161,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int quad = warp & 3;
   const int h = quad * 32 + lane;  // head = TMEM lane owned by this softmax thread
   const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-  if (warp >= 3 && ntiles > 0) {
+  if (warp >= 2 && ntiles > 0) {
     const uint4* src = reinterpret_cast<const uint4*>(p.q + (static_cast<int64_t>(t) * H + h) * kDLat);
 #pragma unroll 1
     for (int c = 0; c < kQTmemDims / 64; ++c) {  // 5 chunks of 64 dims = 32 TMEM columns
@@ -183,55 +186,60 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
 
-  if (warp < 2) {
-    // ---------------- gather producers ----------------
-    const int pt = threadIdx.x;  // 0..63
+  if (warp == 0) {
+    // ---------------- gather producer (TMA gather4; lanes 0..8 own one 64-dim block each) ----------
     bool ok = true;
     for (int it = 0; it < ntiles && ok; ++it) {
       const int s = it % kStages;
-      ok = mbar_wait(&kv_empty[s], ((it / kStages) & 1) ^ 1, p.status, kDevErrTimeout);
+      if (lane == 0) {
+        ok = mbar_wait(&kv_empty[s], ((it / kStages) & 1) ^ 1, p.status, kDevErrTimeout);
+        if (ok) mbar_arrive_expect_tx(&kv_full[s], kTileKeys * kDLat * 2);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      const uint32_t sb = smem_u32(base + MlaSmem::kStage0 + s * kStageBytes);
-      for (int r = pt >> 5; r < kTileKeys; r += 2) {
-        const int e = it * kTileKeys + r;
-        int prow = (e < nkeys) ? rows[e] : -1;
-        if (prow < 0) prow = 0;  // masked in the softmax; any readable row will do
-        const uint8_t* src = reinterpret_cast<const uint8_t*>(p.kv) + static_cast<int64_t>(prow) * (kDLat * 2);
-        const uint32_t dst_row = sb + static_cast<uint32_t>(r * 128);
-        for (int c = lane; c < kDLat * 2 / 16; c += 32) {
-          const uint32_t dst = dst_row + static_cast<uint32_t>((c >> 3) * kBlkBytes) +
-                               (static_cast<uint32_t>((c & 7) ^ (r & 7)) << 4);
-          cp_async_16(dst, src + c * 16);
+      if (lane < kDLat / 64) {
+        uint8_t* dst = base + MlaSmem::kStage0 + s * kStageBytes + lane * kBlkBytes;
+#pragma unroll
+        for (int g = 0; g < kTileKeys / 4; ++g) {
+          int r[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int e = it * kTileKeys + 4 * g + i;
+            r[i] = (e < nkeys) ? rows[e] : -1;
+            if (r[i] < 0) r[i] = 0;  // masked in the softmax; any readable row will do
+          }
+          tma_gather4(dst + g * 512, &kvmap, lane * 64, r[0], r[1], r[2], r[3], &kv_full[s]);
         }
       }
-      cp_async_mbar_arrive_noinc(&kv_full[s]);
     }
-    if (!ok) asm volatile("cp.async.wait_all;" ::: "memory");
-  } else if (warp == 2) {
+  } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0 && ntiles > 0) {
       bool ok = mbar_wait(q_full, 0, p.status, kDevErrTimeout);
       const uint32_t idesc_s = umma_idesc(128, kTileKeys, 1, 0, 0);  // bf16, K-major A and B
       const uint32_t idesc_o = umma_idesc(128, 256, 1, 0, 1);        // bf16, B MN-major
-      const uint32_t q_smem = smem_u32(base + MlaSmem::kQ);
+      // Descriptors are built once; a K step only moves the 14-bit start-address field, so it is a
+      // plain add of a compile-time constant (addresses stay below 256 KB: no carry out of the field).
+      const uint64_t q_desc0 = umma_desc_sw128(smem_u32(base + MlaSmem::kQ), 16, 1024);
+      const uint64_t k_desc0 = umma_desc_sw128(smem_u32(base + MlaSmem::kStage0), 16, 1024);
+      const uint64_t v_desc0 = umma_desc_sw128(smem_u32(base + MlaSmem::kStage0) + 4 * v * kBlkBytes, kBlkBytes, 1024);
       for (int it = 0; it <= ntiles && ok; ++it) {
         if (it < ntiles) {
           const int s = it % kStages, sb = it & 1;
           ok = mbar_wait(&kv_full[s], (it / kStages) & 1, p.status, kDevErrTimeout) &&
                mbar_wait(&s_free[sb], ((it >> 1) & 1) ^ 1, p.status, kDevErrTimeout);
           if (!ok) break;
-          fence_proxy_async_smem();
           tc_fence_after();
-          const uint32_t stage = smem_u32(base + MlaSmem::kStage0 + s * kStageBytes);
+          const uint64_t kd = k_desc0 + static_cast<uint64_t>((s * kStageBytes) >> 4);
           const uint32_t d = tmem + kColS + 32 * sb;
 #pragma unroll
           for (int ks = 0; ks < kDLat / 16; ++ks) {
-            const uint64_t bdesc = umma_desc_sw128(stage + (ks >> 2) * kBlkBytes + (ks & 3) * 32, 16, 1024);
+            const uint64_t bdesc = kd + static_cast<uint64_t>(((ks >> 2) * kBlkBytes + (ks & 3) * 32) >> 4);
             if (ks < kQTmemDims / 16) {
               mma_bf16_ts(d, tmem + kColQ + 8 * ks, bdesc, idesc_s, ks > 0 ? 1u : 0u);
             } else {
               const int qs = ks - kQTmemDims / 16;
-              const uint64_t adesc = umma_desc_sw128(q_smem + (qs >> 2) * kQBlkBytes + (qs & 3) * 32, 16, 1024);
+              const uint64_t adesc = q_desc0 + static_cast<uint64_t>(((qs >> 2) * kQBlkBytes + (qs & 3) * 32) >> 4);
               mma_bf16_ss(d, adesc, bdesc, idesc_s, 1u);
             }
           }
@@ -242,11 +250,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait(&p_full[pb], (i >> 1) & 1, p.status, kDevErrTimeout);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t vbase = smem_u32(base + MlaSmem::kStage0 + s * kStageBytes) + 4 * v * kBlkBytes;
+          const uint64_t vd = v_desc0 + static_cast<uint64_t>((s * kStageBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < kTileKeys / 16; ++kk) {
-            const uint64_t bdesc = umma_desc_sw128(vbase + kk * 2048, kBlkBytes, 1024);
-            mma_bf16_ts(tmem + kColO, tmem + kColP + 16 * pb + 8 * kk, bdesc, idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16_ts(tmem + kColO, tmem + kColP + 16 * pb + 8 * kk, vd + static_cast<uint64_t>((kk * 2048) >> 4),
+                        idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&p_free[pb]);
           mma_commit(&kv_empty[s]);
@@ -256,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ---------------- softmax + epilogue (warps 3..6, one head per thread) ----------------
+    // ---------------- softmax + epilogue (warps 2..5, one head per thread) ----------------
     // l: sum of the fp32 weights (for the log-sum-exp); lr: sum of the bf16-rounded weights the
     // P x V MMA actually uses (normalises O, so the output weights sum to one).
     float m_ref = -INFINITY, l = 0.f, lr = 0.f;
@@ -386,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 2) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -484,15 +492,18 @@ int launch_sparse_mla(const BatchDev& b, const void* plan, const void* q, int H,
   }
   prm.status = &pv.hdr->status;
 
-  CUtensorMap qmap;
+  CUtensorMap qmap, kvmap;
   int e = make_tmap_2d(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, kDLat, static_cast<uint64_t>(b.T) * H,
                        kDLat * 2, 64, 128);
+  if (e) return e;
+  e = make_tmap_2d(&kvmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kv_cache, kDLat,
+                   static_cast<uint64_t>(b.num_pages) * kPage, kDLat * 2, 64, 1);
   if (e) return e;
   cudaError_t ce =
       cudaFuncSetAttribute(sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, MlaSmem::kDynamic);
   if (ce != cudaSuccess) return static_cast<int>(ce);
   dim3 grid(b.T, 2, prm.nsplit);
-  sparse_mla_kernel<<<grid, kThreads, MlaSmem::kDynamic, static_cast<cudaStream_t>(stream)>>>(qmap, prm);
+  sparse_mla_kernel<<<grid, kThreads, MlaSmem::kDynamic, static_cast<cudaStream_t>(stream)>>>(qmap, kvmap, prm);
   ce = cudaGetLastError();
   if (ce != cudaSuccess) return static_cast<int>(ce);
   if (prm.nsplit > 1) {

@@ -4,10 +4,11 @@
 // k = min(L, TOPK) in "MTP 与稀疏注意力：NSA 与 DSA", section "稀疏注意力：NSA 与 DSA").
 //
 // One CTA of 1024 threads per query row. Scores become order-preserving uint32 keys; a radix
-// select over 11 + 11 + 10 bits finds the exact k-th largest key with shared-memory histograms.
-// A last, ordered pass (warp ballots plus a block scan per 1024 positions) emits every position
-// above the threshold and the first `remaining` positions equal to it, in increasing position
-// order, so the result is deterministic: among equal scores the smaller position wins.
+// select over 11 + 11 + 10 bits finds the exact k-th largest key with shared-memory histograms
+// (warp-aggregated atomics: scores crowd into a few exponent bins). A last pass over contiguous
+// per-warp segments (ballot-ordered, two block scans) emits every position above the threshold and
+// the first `remaining` positions equal to it, in increasing position order, so the result is
+// deterministic: among equal scores the smaller position wins.
 // Rows up to kCacheCap scores are kept in shared memory after the first read; longer rows are
 // re-read from L2 on each pass.
 #include <cuda_runtime.h>
@@ -29,6 +30,15 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t b = __float_as_uint(f);
   if (b == 0x80000000u) b = 0u;  // -0 ranks as +0
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// hist[bin] += 1 for every lane, one atomic per distinct bin in the warp (scores cluster in a
+// few exponent bins, so plain per-lane atomics would serialise on them).
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active) {
+  const uint32_t act = __ballot_sync(0xffffffffu, active);
+  if (!active) return;
+  const uint32_t peers = __match_any_sync(act, bin);
+  if ((threadIdx.x & 31) == static_cast<uint32_t>(__ffs(peers) - 1)) atomicAdd(&hist[bin], __popc(peers));
 }
 
 // Block-wide inclusive scan of one value per thread; `scratch` holds kWarps ints.
@@ -87,16 +97,21 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
     const uint32_t bmask = nb - 1u;
     for (uint32_t i = threadIdx.x; i < kBins; i += kThreads) hist[i] = 0u;
     __syncthreads();
+    const int L_pad = (L + 31) & ~31;  // whole warps take part in the aggregated atomics
     if (pass == 0) {
-      for (int j = threadIdx.x; j < L; j += kThreads) {
-        const uint32_t u = order_key(__ldg(row + j));
-        if (cached) cache[j] = u;
-        atomicAdd(&hist[u >> shift], 1u);
+      for (int j = threadIdx.x; j < L_pad; j += kThreads) {
+        uint32_t u = 0;
+        if (j < L) {
+          u = order_key(__ldg(row + j));
+          if (cached) cache[j] = u;
+        }
+        hist_add(hist, u >> shift, j < L);
       }
     } else {
-      for (int j = threadIdx.x; j < L; j += kThreads) {
-        const uint32_t u = cached ? cache[j] : order_key(__ldg(row + j));
-        if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & bmask], 1u);
+      for (int j = threadIdx.x; j < L_pad; j += kThreads) {
+        uint32_t u = 0;
+        if (j < L) u = cached ? cache[j] : order_key(__ldg(row + j));
+        hist_add(hist, (u >> shift) & bmask, j < L && (u & mask) == prefix);
       }
     }
     __syncthreads();
@@ -121,30 +136,43 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
     __syncthreads();
   }
 
-  // ordered emission: keys above the threshold, then the first `remaining` keys equal to it
-  int out_pos = 0;
-  uint32_t ties_seen = 0;
-  const int lane = threadIdx.x & 31;
-  for (int base = 0; base < L; base += kThreads) {
-    const int j = base + threadIdx.x;
-    uint32_t u = 0;
-    if (j < L) u = cached ? cache[j] : order_key(__ldg(row + j));
-    const bool gt = j < L && u > prefix;
-    const bool tie = j < L && u == prefix;
-    int tie_total;
-    const int tie_incl = block_inclusive_scan(tie ? 1 : 0, scan_scratch, &tie_total);
-    const bool sel = gt || (tie && ties_seen + static_cast<uint32_t>(tie_incl - 1) < remaining);
-    int sel_total;
-    const int sel_incl = block_inclusive_scan(sel ? 1 : 0, scan_scratch, &sel_total);
-    if (sel) {
-      const int slot = out_pos + sel_incl - 1;
-      if (slot < k) out[slot] = j;
-    }
-    out_pos += sel_total;
-    ties_seen += static_cast<uint32_t>(tie_total);
-    (void)lane;
+  // Ordered emission. Warp w owns the contiguous positions [w*SEG, (w+1)*SEG), visited 32
+  // consecutive positions at a time (conflict-free, ballot-ordered). Two block scans over the
+  // per-warp counts rank the ties (the first `remaining` in position order are taken) and give
+  // each warp its output offset.
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const int SEG = 32 * ((L + kThreads - 1) / kThreads);
+  const int wj0 = min(L, wid * SEG), wj1 = min(L, wj0 + SEG);
+  int w_gt = 0, w_tie = 0;
+  for (int base = wj0; base < wj1; base += 32) {
+    const int j = base + lane;
+    const uint32_t u = (j < wj1) ? (cached ? cache[j] : order_key(__ldg(row + j))) : 0u;
+    w_gt += __popc(__ballot_sync(0xffffffffu, j < wj1 && u > prefix));
+    w_tie += __popc(__ballot_sync(0xffffffffu, j < wj1 && u == prefix));
   }
-  for (int s = out_pos + static_cast<int>(threadIdx.x); s < k; s += kThreads) out[s] = -1;
+  int total;
+  const int tie_incl = __shfl_sync(0xffffffffu, block_inclusive_scan(lane == 0 ? w_tie : 0, scan_scratch, &total), 0);
+  const int tie_take = max(0, min(w_tie, static_cast<int>(remaining) - (tie_incl - w_tie)));
+  const int sel = w_gt + tie_take;
+  const int sel_incl = __shfl_sync(0xffffffffu, block_inclusive_scan(lane == 0 ? sel : 0, scan_scratch, &total), 0);
+  int slot = sel_incl - sel, ties_left = tie_take;
+  for (int base = wj0; base < wj1; base += 32) {
+    const int j = base + lane;
+    const uint32_t u = (j < wj1) ? (cached ? cache[j] : order_key(__ldg(row + j))) : 0u;
+    const bool gt = j < wj1 && u > prefix;
+    const bool tie = j < wj1 && u == prefix;
+    const uint32_t tie_mask = __ballot_sync(0xffffffffu, tie);
+    const bool take = gt || (tie && __popc(tie_mask & lt_mask) < ties_left);
+    const uint32_t take_mask = __ballot_sync(0xffffffffu, take);
+    if (take) {
+      const int o = slot + __popc(take_mask & lt_mask);
+      if (o < k) out[o] = j;
+    }
+    slot += __popc(take_mask);
+    ties_left -= min(__popc(tie_mask), ties_left);
+  }
+  for (int s2 = total + static_cast<int>(threadIdx.x); s2 < k; s2 += kThreads) out[s2] = -1;
 }
 
 }  // namespace
