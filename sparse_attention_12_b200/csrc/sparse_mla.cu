@@ -7,23 +7,32 @@
 // 576-wide latent shared by all heads per "MTP 与稀疏注意力：NSA 与 DSA", section "稀疏注意力：NSA 与
 // DSA". S_t is shared by all heads.)
 //
-// One CTA per (query row, half of the 512 value dims, split of S_t); one CTA per SM.
-//   * Q (128 heads x 576, bf16): dims 0..319 sit in TMEM and feed the S = Q C^T MMAs as the A
-//     operand; dims 320..575 sit in shared memory (TMA, 128-byte swizzle).
-//   * Latent rows c_j are gathered 32 at a time through the block table with TMA tile::gather4
-//     (4 rows x 64 dims per copy, 72 copies per tile) into a 4-stage ring; the tensor map's 128-byte
-//     swizzle follows the shared-memory address, so 4-row copies at 512-byte steps build the
-//     canonical K-major UMMA layout (9 blocks of 64 dims, 8-row atoms).
-//   * S tile [128 heads x 32 keys] accumulates in TMEM (double-buffered), the softmax warps turn it
-//     into P (bf16) in TMEM, and O[:, half] (128 x 256 fp32) accumulates in TMEM from P x V with
-//     V read from the same shared-memory stage in its MN-major view.
-//   * Online softmax with lazy rescaling: the reference maximum only moves when a tile's maximum
-//     exceeds it by more than 2^8, so O is rarely touched outside the MMAs.
-// TMEM columns: O 0..255 | S 256..319 (2 x 32) | P 320..351 (2 x 16) | Q 352..511 (160).
-// Warps: 0 gather producer (TMA), 1 MMA issuer (+ TMEM allocator), 2-5 softmax and epilogue.
+// One cluster of two CTAs (on two SMs) per (query row, split of S_t):
 //
-// Splits (several CTAs over one S_t) write normalised partial outputs and their log-sum-exp to the
-// workspace; a combine kernel merges them: o = sum_s exp(lse_s - lse) o_s.
+//   S-CTA (rank 0): S = Q C^T and the softmax.
+//     * Q (128 heads x 576 bf16): dims 0..511 in TMEM as the A operand (256 columns), the 64 rope
+//       dims in shared memory (one 128-byte-swizzled block).
+//     * The selected latent rows are gathered by 16 producer warps with 16-byte cp.async (8 lanes
+//       per 128-byte row segment, XOR-swizzled on the way into the canonical 128-byte-swizzled
+//       K-major UMMA layout) into a 12-slot ring of 128 keys x 64 dims. Random 1152-byte rows need
+//       hundreds of loads in flight per SM; TMA gather4 tops out near 2 TB/s here (per-copy cost).
+//     * Each tile of 128 keys costs 36 tcgen05.mma (M=128 heads, N=128 keys, K=16), which run at
+//       the full bf16 rate; S tiles are double-buffered in TMEM (2 x 128 columns).
+//     * Four softmax warps (thread = head) read each S tile twice from TMEM (maximum, then
+//       exponentials, to keep registers low) and turn it into P (bf16) with an online softmax whose
+//       reference maximum only moves when a tile's maximum exceeds it by more than 2^8, and store
+//       P, the per-head rescale factor and a per-warp "rescale" flag straight into the O-CTA's
+//       shared memory (distributed shared memory), then arrive on the O-CTA's barrier.
+//   O-CTA (rank 1): O = P V.
+//     * O (128 heads x 512 fp32) fills its whole TMEM. V = c[0:512] of the same rows is gathered
+//       by its own 16 producer warps in units of 128 keys x 128 dims (4 per tile).
+//     * Per tile: 32 tcgen05.mma (M=128, N=128 dims, K=16 keys), A = P (shared memory, K-major),
+//       B = V (MN-major). Completion is multicast back to the S-CTA to free the P buffer.
+//     * Four correction warps rescale O rows in TMEM when the S-CTA flags a new reference
+//       maximum (rare), and at the end normalise O and write the output.
+//
+// Splits (several clusters over one S_t) write normalised partial outputs and their log-sum-exp
+// to the workspace; a combine kernel merges them: o = sum_s exp(lse_s - lse) o_s.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -39,42 +48,84 @@ int make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, co
 
 namespace {
 
-constexpr int kTileKeys = 32;
-constexpr int kStages = 4;
-constexpr int kBlkBytes = kTileKeys * 128;           // one 64-dim block of a tile: 4 KB
-constexpr int kStageBytes = 9 * kBlkBytes;           // 36 KB
-constexpr int kQTmemDims = 320;                      // Q dims held in TMEM
-constexpr int kQSmemBlocks = (kDLat - kQTmemDims) / 64;  // 4 blocks in shared memory
-constexpr int kQBlkBytes = 128 * 128;                // 16 KB
-constexpr int kMaxKeysPerCta = 2048;
-constexpr int kThreads = 192;
-constexpr float kRescaleThreshold = 8.0f;            // log2 units
+using kv_t = uint8_t;
+constexpr int kRowBytes = kDLat * 2;         // 1152
+constexpr int kTile = 128;                   // keys per tile (MMA N for S, K-extent for P V)
+constexpr int kMaxKeysPerCta = 2048;         // S_t entries one cluster handles
+constexpr int kMaxTiles = kMaxKeysPerCta / kTile;
+constexpr int kBlk = kTile * 128;            // 128 keys x 64 dims bf16 = 16 KB
+constexpr int kKSlots = 12;                  // S-CTA ring slots (one 64-dim block of one tile each)
+constexpr int kVSlots = 4;                   // O-CTA ring slots (two 64-dim blocks of one tile each)
+constexpr int kProdWarps = 16;               // warps 0..15: gather producers
+constexpr int kGroupWarps = 4;               // warps per producer group (one ring unit per group)
+constexpr int kGroups = kProdWarps / kGroupWarps;
+constexpr int kMmaWarp = kProdWarps;         // warp 16: TMEM allocator and MMA issuer
+constexpr int kSoftWarp0 = kProdWarps + 1;   // warps 17..20: softmax (S-CTA) / correction (O-CTA)
+constexpr int kThreads = 32 * (kProdWarps + 5);
+constexpr float kRescaleThreshold = 8.0f;    // log2 units
 
-constexpr uint32_t kColO = 0, kColS = 256, kColP = 320, kColQ = 352;
+// TMEM columns
+constexpr uint32_t kColS = 0;      // S-CTA: S tiles at 0 and 128
+constexpr uint32_t kColQ = 256;    // S-CTA: Q dims 0..511
+constexpr uint32_t kColO = 0;      // O-CTA: O, 512 columns
 
-struct MlaSmem {
-  static constexpr int kQ = 0;
-  static constexpr int kStage0 = kQ + kQSmemBlocks * kQBlkBytes;      // 64 KB
-  static constexpr int kRows = kStage0 + kStages * kStageBytes;        // 208 KB
-  static constexpr int kBars = kRows + kMaxKeysPerCta * 4;             // 216 KB
-  static constexpr int kNumBars = 2 * kStages + 2 + 2 + 2 + 2 + 1 + 1;
+struct Smem {
+  // S-CTA
+  static constexpr int kQRope = 0;                               // 16 KB
+  static constexpr int kKRing = kQRope + kBlk;                   // 12 x 16 KB
+  static constexpr int kSEnd = kKRing + kKSlots * kBlk;          // 208 KB
+  // O-CTA
+  static constexpr int kP = 0;                                   // 2 x 32 KB
+  static constexpr int kVRing = kP + 2 * 2 * kBlk;               // 4 x 32 KB
+  static constexpr int kAlpha = kVRing + kVSlots * 2 * kBlk;     // float [2][128]
+  static constexpr int kFlags = kAlpha + 2 * 128 * 4;            // u32 [2][4]
+  static constexpr int kStats = kFlags + 2 * 4 * 4;              // float [3][128]: m, l, lr
+  static constexpr int kOEnd = kStats + 3 * 128 * 4;
+  // both
+  static constexpr int kCommon = (kSEnd > kOEnd ? kSEnd : kOEnd);
+  static constexpr int kRows = kCommon;                          // int32 [2048] physical rows
+  static constexpr int kMasks = kRows + kMaxKeysPerCta * 4;      // u32 [16][4] validity bits
+  static constexpr int kBars = kMasks + kMaxTiles * 4 * 4;
+  static constexpr int kNumBars = 64;
   static constexpr int kTmemSlot = kBars + kNumBars * 8;
   static constexpr int kTotal = kTmemSlot + 16;
   static constexpr int kDynamic = kTotal + 1024;
 };
-static_assert(MlaSmem::kDynamic <= 232448, "sparse MLA shared memory exceeds the 227 KB limit");
+static_assert(Smem::kDynamic <= 232448, "sparse MLA shared memory exceeds the 227 KB limit");
+
+// barrier indices (same offsets in both CTAs; each CTA initialises the ones it owns)
+enum : int {
+  // S-CTA
+  B_KFULL = 0,                      // [12]
+  B_KEMPTY = B_KFULL + kKSlots,     // [12]
+  B_QROPE = B_KEMPTY + kKSlots,     // 1
+  B_SFULL = B_QROPE + 1,            // [2]  MMA -> softmax
+  B_SFREE = B_SFULL + 2,            // [2]  softmax -> MMA (4 warps)
+  B_PFREE = B_SFREE + 2,            // [2]  O-CTA MMA -> S-CTA softmax (multicast commit)
+  B_QCONS = B_PFREE + 2,            // 1    softmax warps have moved Q out of the ring (4 warps)
+  // O-CTA
+  B_VFULL = B_QCONS + 1,            // [4]
+  B_VEMPTY = B_VFULL + kVSlots,     // [4]
+  B_PFULL = B_VEMPTY + kVSlots,     // [2]  S-CTA softmax -> O-CTA (128 remote arrivals)
+  B_OREADY = B_PFULL + 2,           // [2]  correction warps -> MMA (4 warps)
+  B_ODONE = B_OREADY + 2,           // 1    MMA -> correction warps (once per tile)
+  B_OFINAL = B_ODONE + 1,           // 1    MMA -> epilogue (once, after the last tile)
+  B_STATS = B_OFINAL + 1,           // 1    S-CTA softmax -> O-CTA epilogue (128 remote arrivals)
+  B_COUNT = B_STATS + 1
+};
+static_assert(B_COUNT <= Smem::kNumBars, "barrier space");
 
 struct MlaParams {
   BatchDev bd;
   const int32_t* row_req;
   const int32_t* row_pos;
   const uint16_t* q;
-  const uint16_t* kv;
+  const uint8_t* kv;  // latent cache, rows of 1152 bytes
   const int32_t* S;
   int k;
   int H;
   int nsplit;
-  int chunk;          // S_t entries per split (multiple of 32)
+  int chunk;          // S_t entries per split (multiple of kTile)
   float scale_log2;   // softmax scale * log2(e)
   uint16_t* out;
   float* lse;
@@ -83,318 +134,431 @@ struct MlaParams {
   uint32_t* status;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
-    sparse_mla_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kvmap,
-                      const MlaParams p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    sparse_mla_kernel(const __grid_constant__ CUtensorMap qmap, const MlaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  int32_t* rows = reinterpret_cast<int32_t*>(base + MlaSmem::kRows);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + MlaSmem::kBars);
-  uint64_t* kv_full = bars;
-  uint64_t* kv_empty = bars + kStages;
-  uint64_t* s_full = bars + 2 * kStages;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_free + 2;
-  uint64_t* p_free = p_full + 2;
-  uint64_t* o_full = p_free + 2;
-  uint64_t* q_full = o_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + MlaSmem::kTmemSlot);
+  int32_t* rows = reinterpret_cast<int32_t*>(base + Smem::kRows);
+  uint32_t* masks = reinterpret_cast<uint32_t*>(base + Smem::kMasks);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(base + Smem::kBars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + Smem::kTmemSlot);
 
+  const uint32_t rank = cluster_ctarank();
+  const bool is_s = rank == 0;
   const int warp = warp_id(), lane = lane_id();
-  const int t = blockIdx.x, v = blockIdx.y, split = blockIdx.z;
+  const int unit = blockIdx.x >> 1;
+  const int t = unit / p.nsplit, split = unit % p.nsplit;
   const int H = p.H;
   const int b = __ldg(p.row_req + t);
   const int pos = __ldg(p.row_pos + t);
-  const int nvis = min(p.k, pos + 1);                 // entries of S_t that can be valid
+  const int nvis = min(p.k, pos + 1);
   const int e0 = split * p.chunk;
-  const int nkeys = max(0, min(nvis - e0, p.chunk));  // entries this CTA reads
-  const int ntiles = (nkeys + kTileKeys - 1) / kTileKeys;
+  const int nkeys = max(0, min(nvis - e0, p.chunk));
+  const int ntiles = (nkeys + kTile - 1) / kTile;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+    if (is_s) {
+      for (int i = 0; i < kKSlots; ++i) {
+        mbar_init(&bar[B_KFULL + i], 32 * kGroupWarps);  // one cp.async arrival per producer lane
+        mbar_init(&bar[B_KEMPTY + i], 1);
+      }
+      mbar_init(&bar[B_QROPE], 1);
+      mbar_init(&bar[B_QCONS], 4);
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&bar[B_SFULL + i], 1);
+        mbar_init(&bar[B_SFREE + i], 4);
+        mbar_init(&bar[B_PFREE + i], 1);
+      }
+    } else {
+      for (int i = 0; i < kVSlots; ++i) {
+        mbar_init(&bar[B_VFULL + i], 32 * kGroupWarps);
+        mbar_init(&bar[B_VEMPTY + i], 1);
+      }
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&bar[B_PFULL + i], 128);
+        mbar_init(&bar[B_OREADY + i], 4);
+      }
+      mbar_init(&bar[B_ODONE], 1);
+      mbar_init(&bar[B_OFINAL], 1);
+      mbar_init(&bar[B_STATS], 128);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
-      mbar_init(&p_full[i], 4);
-      mbar_init(&p_free[i], 1);
-    }
-    mbar_init(o_full, 1);
-    mbar_init(q_full, 1);
     fence_barrier_init();
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
+  }
+
+  // physical rows of this cluster's entries (both CTAs); -1 marks an entry to skip
+  const int32_t* S_row = p.S + static_cast<int64_t>(t) * p.k + e0;
+  const int32_t* bt_row = p.bd.block_table + static_cast<int64_t>(b) * p.bd.max_pages;
+  const int n_b = __ldg(p.bd.seq_lens + b);
+  for (int e = threadIdx.x; e < ntiles * kTile; e += kThreads) {
+    int r = -1;
+    if (e < nkeys) {
+      const int j = __ldg(S_row + e);
+      if (j >= 0) {
+        if (j > pos || j >= n_b) {
+          report_error(p.status, kDevErrIndex);
+        } else {
+          const int pg = __ldg(bt_row + j / kPage);
+          if (pg < 0 || pg >= p.bd.num_pages)
+            report_error(p.status, kDevErrIndex);
+          else
+            r = pg * kPage + (j % kPage);
+        }
+      }
+    }
+    rows[e] = r;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  // ---- set-up: physical rows of this CTA's entries, Q into shared memory and TMEM ----------
-  const int32_t* S_row = p.S + static_cast<int64_t>(t) * p.k + e0;
-  const int32_t* bt_row = p.bd.block_table + static_cast<int64_t>(b) * p.bd.max_pages;
-  const int n_b = __ldg(p.bd.seq_lens + b);
-  for (int e = threadIdx.x; e < nkeys; e += kThreads) {
-    const int j = __ldg(S_row + e);
-    int r = -1;
-    if (j >= 0) {
-      if (j > pos || j >= n_b) {
-        report_error(p.status, kDevErrIndex);
-      } else {
-        const int pg = __ldg(bt_row + j / kPage);
-        if (pg < 0 || pg >= p.bd.num_pages)
-          report_error(p.status, kDevErrIndex);
-        else
-          r = pg * kPage + (j % kPage);
-      }
-    }
-    rows[e] = r;
-  }
-  if (threadIdx.x == 0 && ntiles > 0) {
-    tma_prefetch_desc(&qmap);
-    tma_prefetch_desc(&kvmap);
-    mbar_arrive_expect_tx(q_full, kQSmemBlocks * kQBlkBytes);
-    for (int i = 0; i < kQSmemBlocks; ++i)
-      tma_load_2d(base + MlaSmem::kQ + i * kQBlkBytes, &qmap, kQTmemDims + 64 * i, t * H, q_full);
-  }
   const int quad = warp & 3;
-  const int h = quad * 32 + lane;  // head = TMEM lane owned by this softmax thread
+  const int h = quad * 32 + lane;
   const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-  if (warp >= 2 && ntiles > 0) {
-    const uint4* src = reinterpret_cast<const uint4*>(p.q + (static_cast<int64_t>(t) * H + h) * kDLat);
-#pragma unroll 1
-    for (int c = 0; c < kQTmemDims / 64; ++c) {  // 5 chunks of 64 dims = 32 TMEM columns
-      uint32_t r[32];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        uint4 x = make_uint4(0, 0, 0, 0);
-        if (h < H) x = __ldg(src + c * 8 + i);
-        r[4 * i + 0] = x.x;
-        r[4 * i + 1] = x.y;
-        r[4 * i + 2] = x.z;
-        r[4 * i + 3] = x.w;
-      }
-      tmem_st32(tmem + lane_base + kColQ + 32 * c, r);
+
+  if (is_s) {
+    if (static_cast<int>(threadIdx.x) < ntiles * 4) {  // mask word w of tile i covers keys 32w..32w+31
+      const int i = threadIdx.x >> 2, w = threadIdx.x & 3;
+      uint32_t m = 0;
+      for (int c = 0; c < 32; ++c) m |= (rows[i * kTile + 32 * w + c] >= 0 ? 1u : 0u) << c;
+      masks[threadIdx.x] = m;
     }
-    tmem_wait_st();
+    if (threadIdx.x == 0 && ntiles > 0) {  // Q: 9 boxes of 128 heads x 64 dims (rope -> its own slot)
+      tma_prefetch_desc(&qmap);
+      mbar_arrive_expect_tx(&bar[B_QROPE], 9 * kBlk);
+      for (int blk = 0; blk < 8; ++blk)
+        tma_load_2d(base + Smem::kKRing + blk * kBlk, &qmap, 64 * blk, t * H, &bar[B_QROPE]);
+      tma_load_2d(base + Smem::kQRope, &qmap, 512, t * H, &bar[B_QROPE]);
+    }
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // barriers of both CTAs initialised before any remote arrival
   tc_fence_after();
 
-  if (warp == 0) {
-    // ---------------- gather producer (TMA gather4; lanes 0..8 own one 64-dim block each) ----------
-    bool ok = true;
-    for (int it = 0; it < ntiles && ok; ++it) {
-      const int s = it % kStages;
-      if (lane == 0) {
-        ok = mbar_wait(&kv_empty[s], ((it / kStages) & 1) ^ 1, p.status, kDevErrTimeout);
-        if (ok) mbar_arrive_expect_tx(&kv_full[s], kTileKeys * kDLat * 2);
+  if (is_s) {
+    if (warp < kProdWarps) {
+      // ---------- S-CTA producers: group g fills units g, g+4, ... (128 keys x 64 dims each) ----------
+      // lane l of warp w of the group copies 16-byte chunk (l & 7) of rows 4j + (l >> 3) + 32 w'
+      const int g = warp / kGroupWarps, wg = warp % kGroupWarps;
+      bool ok = ntiles == 0 || mbar_wait(&bar[B_QCONS], 0, p.status, kDevErrTimeout);
+      const kv_t* kv = p.kv;
+      for (int u = g; u < ntiles * 9 && ok; u += kGroups) {
+        const int i = u / 9, blk = u % 9, slot = u % kKSlots;
+        ok = mbar_wait(&bar[B_KEMPTY + slot], ((u / kKSlots) & 1) ^ 1, p.status, kDevErrTimeout);
+        if (!ok) break;
+        const uint32_t sbase = smem_u32(base + Smem::kKRing + slot * kBlk);
+        const int c = lane & 7;
+#pragma unroll 4
+        for (int j = 0; j < kTile / (4 * kGroupWarps); ++j) {
+          const int r = (wg * (kTile / kGroupWarps)) + 4 * j + (lane >> 3);
+          const int prow = max(rows[i * kTile + r], 0);
+          cp_async_16(sbase + r * 128 + (((c ^ (r & 7))) << 4), kv + static_cast<int64_t>(prow) * kRowBytes + blk * 128 + c * 16);
+        }
+        cp_async_mbar_arrive_noinc(&bar[B_KFULL + slot]);
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      if (lane < kDLat / 64) {
-        uint8_t* dst = base + MlaSmem::kStage0 + s * kStageBytes + lane * kBlkBytes;
+      if (!ok) asm volatile("cp.async.wait_all;" ::: "memory");
+    } else if (warp == kMmaWarp) {
+      // ---------- S-CTA MMA issuer: S[h, key] = Q . C^T over 9 blocks of 64 dims ----------
+      if (lane == 0 && ntiles > 0) {
+        // Q rope in shared memory (TMA) and Q dims 0..511 in TMEM (softmax warps) before the first MMA
+        bool ok = mbar_wait(&bar[B_QROPE], 0, p.status, kDevErrTimeout) &&
+                  mbar_wait(&bar[B_QCONS], 0, p.status, kDevErrTimeout);
+        tc_fence_after();
+        const uint32_t idesc = umma_idesc(128, kTile, 1, 0, 0);
+        const uint64_t kdesc0 = umma_desc_sw128(smem_u32(base + Smem::kKRing), 16, 1024);
+        const uint64_t rdesc = umma_desc_sw128(smem_u32(base + Smem::kQRope), 16, 1024);
+        for (int i = 0; i < ntiles && ok; ++i) {
+          const int sb = i & 1;
+          ok = mbar_wait(&bar[B_SFREE + sb], ((i >> 1) & 1) ^ 1, p.status, kDevErrTimeout);
+          if (!ok) break;
+          const uint32_t d = tmem + kColS + kTile * sb;
+          for (int blk = 0; blk < 9; ++blk) {
+            const int u = i * 9 + blk, slot = u % kKSlots;
+            ok = mbar_wait(&bar[B_KFULL + slot], (u / kKSlots) & 1, p.status, kDevErrTimeout);
+            if (!ok) break;
+            fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tensor-core reads
+            tc_fence_after();
+            const uint64_t bd = kdesc0 + static_cast<uint64_t>((slot * kBlk) >> 4);
+            if (blk < 8) {
 #pragma unroll
-        for (int g = 0; g < kTileKeys / 4; ++g) {
-          int r[4];
+              for (int kk = 0; kk < 4; ++kk)
+                mma_bf16_ts(d, tmem + kColQ + 32 * blk + 8 * kk, bd + 2 * kk, idesc, (blk | kk) ? 1u : 0u);
+            } else {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int e = it * kTileKeys + 4 * g + i;
-            r[i] = (e < nkeys) ? rows[e] : -1;
-            if (r[i] < 0) r[i] = 0;  // masked in the softmax; any readable row will do
+              for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(d, rdesc + 2 * kk, bd + 2 * kk, idesc, 1u);
+            }
+            mma_commit(&bar[B_KEMPTY + slot]);
           }
-          tma_gather4(dst + g * 512, &kvmap, lane * 64, r[0], r[1], r[2], r[3], &kv_full[s]);
+          if (!ok) break;
+          mma_commit(&bar[B_SFULL + sb]);
         }
       }
+      __syncwarp();
+    } else {
+      // ---------- S-CTA softmax (warps 17..20, thread = head) ----------
+      const uint32_t peer_p = peer_addr(smem_u32(base + Smem::kP), 1);
+      const uint32_t peer_alpha = peer_addr(smem_u32(base + Smem::kAlpha), 1);
+      const uint32_t peer_flags = peer_addr(smem_u32(base + Smem::kFlags), 1);
+      const uint32_t peer_stats = peer_addr(smem_u32(base + Smem::kStats), 1);
+      const uint32_t peer_pfull = peer_addr(smem_u32(&bar[B_PFULL]), 1);
+      const uint32_t peer_statbar = peer_addr(smem_u32(&bar[B_STATS]), 1);
+      float m_ref = -INFINITY, l = 0.f, lr = 0.f;
+      bool ok = true;
+      if (ntiles > 0) {
+        // Q dims 0..511: 8 swizzled blocks in ring slots 0..7 -> TMEM columns 256..511 (lane = head)
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_QROPE], 0, p.status, kDevErrTimeout));
+        if (ok) {
+          for (int blk = 0; blk < 8; ++blk) {
+            const uint8_t* rowp = base + Smem::kKRing + blk * kBlk + h * 128;
+            uint32_t r[32];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const uint4 x = (h < H) ? *reinterpret_cast<const uint4*>(rowp + ((c ^ (h & 7)) << 4)) : make_uint4(0, 0, 0, 0);
+              r[4 * c + 0] = x.x;
+              r[4 * c + 1] = x.y;
+              r[4 * c + 2] = x.z;
+              r[4 * c + 3] = x.w;
+            }
+            tmem_st32(tmem + lane_base + kColQ + 32 * blk, r);
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[B_QCONS]);  // ring slots 0..7 may be refilled
+      }
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const int sb = i & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_SFULL + sb], (i >> 1) & 1, p.status, kDevErrTimeout));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t srow = tmem + lane_base + kColS + kTile * sb;
+        // pass 1: tile maximum (scaled, log2 units) over the valid keys
+        float tmax = -INFINITY;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld32_sync(srow + 32 * c, v);
+          const uint32_t m = masks[4 * i + c];
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if ((m >> j) & 1u) tmax = fmaxf(tmax, __uint_as_float(v[j]) * p.scale_log2);
+        }
+        const bool need = tmax > m_ref + kRescaleThreshold;
+        const float alpha = need ? exp2f(m_ref - tmax) : 1.f;  // 0 when m_ref is -inf
+        if (need) {
+          l *= alpha;
+          lr *= alpha;
+          m_ref = tmax;
+        }
+        const bool warp_rescale = __any_sync(0xffffffffu, need && i > 0);
+        // the O-CTA must be done with the P buffer of tile i-2
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_PFREE + sb], ((i >> 1) & 1) ^ 1, p.status, kDevErrTimeout));
+        if (!ok) break;
+        // pass 2: P row h (128 keys, bf16) into the peer's K-major swizzled buffer (2 blocks of 64)
+        const uint32_t prow = peer_p + static_cast<uint32_t>(sb * 2 * kBlk + h * 128);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld32_sync(srow + 32 * c, v);
+          const uint32_t m = masks[4 * i + c];
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {  // 8 keys = one 16-byte chunk
+            uint32_t w[4];
+#pragma unroll
+            for (int q2 = 0; q2 < 4; ++q2) {
+              const int j0 = 8 * q8 + 2 * q2;
+              const float p0 = ((m >> j0) & 1u) && m_ref > -INFINITY
+                                   ? exp2f(__uint_as_float(v[j0]) * p.scale_log2 - m_ref) : 0.f;
+              const float p1 = ((m >> (j0 + 1)) & 1u) && m_ref > -INFINITY
+                                   ? exp2f(__uint_as_float(v[j0 + 1]) * p.scale_log2 - m_ref) : 0.f;
+              const __nv_bfloat162 bp = __floats2bfloat162_rn(p0, p1);
+              l += p0 + p1;
+              lr += __low2float(bp) + __high2float(bp);
+              w[q2] = *reinterpret_cast<const uint32_t*>(&bp);
+            }
+            const int chunk = 4 * c + q8;  // 0..15: block chunk>>3, chunk-in-block chunk&7
+            const uint32_t addr = prow + static_cast<uint32_t>((chunk >> 3) * kBlk + (((chunk & 7) ^ (h & 7)) << 4));
+            st_cluster_v4(addr, w[0], w[1], w[2], w[3]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[B_SFREE + sb]);
+        st_cluster_f32(peer_alpha + static_cast<uint32_t>((sb * 128 + h) * 4), alpha);
+        if (lane == 0) st_cluster_u32(peer_flags + static_cast<uint32_t>((sb * 4 + quad) * 4), warp_rescale ? 1u : 0u);
+        fence_proxy_async_cluster();
+        mbar_arrive_remote(peer_pfull + static_cast<uint32_t>(sb * 8));
+      }
+      // final statistics for the epilogue, always sent so the O-CTA never waits in vain
+      st_cluster_f32(peer_stats + static_cast<uint32_t>(h * 4), m_ref);
+      st_cluster_f32(peer_stats + static_cast<uint32_t>((128 + h) * 4), l);
+      st_cluster_f32(peer_stats + static_cast<uint32_t>((256 + h) * 4), lr);
+      mbar_arrive_remote(peer_statbar);
+      // the last multicast commits of the O-CTA land in this CTA's barriers: wait for them
+      if (ok && ntiles > 0) {
+        const int i1 = ntiles - 1;
+        mbar_wait(&bar[B_PFREE + (i1 & 1)], (i1 >> 1) & 1, p.status, kDevErrTimeout);
+        if (ntiles > 1) mbar_wait(&bar[B_PFREE + ((i1 - 1) & 1)], ((i1 - 1) >> 1) & 1, p.status, kDevErrTimeout);
+      }
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0 && ntiles > 0) {
-      bool ok = mbar_wait(q_full, 0, p.status, kDevErrTimeout);
-      const uint32_t idesc_s = umma_idesc(128, kTileKeys, 1, 0, 0);  // bf16, K-major A and B
-      const uint32_t idesc_o = umma_idesc(128, 256, 1, 0, 1);        // bf16, B MN-major
-      // Descriptors are built once; a K step only moves the 14-bit start-address field, so it is a
-      // plain add of a compile-time constant (addresses stay below 256 KB: no carry out of the field).
-      const uint64_t q_desc0 = umma_desc_sw128(smem_u32(base + MlaSmem::kQ), 16, 1024);
-      const uint64_t k_desc0 = umma_desc_sw128(smem_u32(base + MlaSmem::kStage0), 16, 1024);
-      const uint64_t v_desc0 = umma_desc_sw128(smem_u32(base + MlaSmem::kStage0) + 4 * v * kBlkBytes, kBlkBytes, 1024);
-      for (int it = 0; it <= ntiles && ok; ++it) {
-        if (it < ntiles) {
-          const int s = it % kStages, sb = it & 1;
-          ok = mbar_wait(&kv_full[s], (it / kStages) & 1, p.status, kDevErrTimeout) &&
-               mbar_wait(&s_free[sb], ((it >> 1) & 1) ^ 1, p.status, kDevErrTimeout);
+  } else {
+    if (warp < kProdWarps) {
+      // ---------- O-CTA producers: V in units of 128 keys x 128 dims (2 blocks), one unit per group ----
+      // lane l copies 16-byte chunk (l & 15) of rows 2j + (l >> 4) of its warp's quarter of the unit
+      const int g = warp / kGroupWarps, wg = warp % kGroupWarps;
+      const kv_t* kv = p.kv;
+      bool ok = true;
+      for (int u = g; u < ntiles * 4 && ok; u += kGroups) {
+        const int i = u / 4, qd = u % 4, slot = u % kVSlots;
+        ok = mbar_wait(&bar[B_VEMPTY + slot], ((u / kVSlots) & 1) ^ 1, p.status, kDevErrTimeout);
+        if (!ok) break;
+        const uint32_t sbase = smem_u32(base + Smem::kVRing + slot * 2 * kBlk);
+        const int c = lane & 15;
+#pragma unroll 4
+        for (int j = 0; j < kTile / (2 * kGroupWarps); ++j) {
+          const int r = (wg * (kTile / kGroupWarps)) + 2 * j + (lane >> 4);
+          const int prow = max(rows[i * kTile + r], 0);
+          cp_async_16(sbase + (c >> 3) * kBlk + r * 128 + (((c & 7) ^ (r & 7)) << 4),
+                      kv + static_cast<int64_t>(prow) * kRowBytes + qd * 256 + c * 16);
+        }
+        cp_async_mbar_arrive_noinc(&bar[B_VFULL + slot]);
+      }
+      if (!ok) asm volatile("cp.async.wait_all;" ::: "memory");
+    } else if (warp == kMmaWarp) {
+      // ---------- O-CTA MMA issuer: O[:, 128qd..] += P . V[:, 128qd..] ----------
+      if (lane == 0 && ntiles > 0) {
+        const uint32_t idesc = umma_idesc(128, 128, 1, 0, 1);  // bf16, A K-major, B MN-major
+        const uint64_t pdesc0 = umma_desc_sw128(smem_u32(base + Smem::kP), 16, 1024);
+        const uint64_t vdesc0 = umma_desc_sw128(smem_u32(base + Smem::kVRing), kBlk, 1024);
+        bool ok = true;
+        for (int i = 0; i < ntiles && ok; ++i) {
+          const int pb = i & 1;
+          ok = mbar_wait(&bar[B_OREADY + pb], (i >> 1) & 1, p.status, kDevErrTimeout) &&
+               mbar_wait_cluster(&bar[B_PFULL + pb], (i >> 1) & 1, p.status, kDevErrTimeout);
           if (!ok) break;
           tc_fence_after();
-          const uint64_t kd = k_desc0 + static_cast<uint64_t>((s * kStageBytes) >> 4);
-          const uint32_t d = tmem + kColS + 32 * sb;
+          const uint64_t pd = pdesc0 + static_cast<uint64_t>((pb * 2 * kBlk) >> 4);
+          for (int qd = 0; qd < 4; ++qd) {
+            const int u = i * 4 + qd, slot = u % kVSlots;
+            ok = mbar_wait(&bar[B_VFULL + slot], (u / kVSlots) & 1, p.status, kDevErrTimeout);
+            if (!ok) break;
+            fence_proxy_async_smem();
+            tc_fence_after();
+            const uint64_t vd = vdesc0 + static_cast<uint64_t>((slot * 2 * kBlk) >> 4);
 #pragma unroll
-          for (int ks = 0; ks < kDLat / 16; ++ks) {
-            const uint64_t bdesc = kd + static_cast<uint64_t>(((ks >> 2) * kBlkBytes + (ks & 3) * 32) >> 4);
-            if (ks < kQTmemDims / 16) {
-              mma_bf16_ts(d, tmem + kColQ + 8 * ks, bdesc, idesc_s, ks > 0 ? 1u : 0u);
-            } else {
-              const int qs = ks - kQTmemDims / 16;
-              const uint64_t adesc = q_desc0 + static_cast<uint64_t>(((qs >> 2) * kQBlkBytes + (qs & 3) * 32) >> 4);
-              mma_bf16_ss(d, adesc, bdesc, idesc_s, 1u);
+            for (int kk = 0; kk < kTile / 16; ++kk) {
+              const uint64_t ad = pd + static_cast<uint64_t>(((kk >> 2) * kBlk + (kk & 3) * 32) >> 4);
+              mma_bf16_ss(tmem + kColO + 128 * qd, ad, vd + static_cast<uint64_t>((kk * 2048) >> 4), idesc,
+                          (i > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&bar[B_VEMPTY + slot]);
+          }
+          if (!ok) break;
+          mma_commit(&bar[B_ODONE]);
+          if (i == ntiles - 1) mma_commit(&bar[B_OFINAL]);
+          mma_commit_multicast(&bar[B_PFREE + pb], 1);  // to the S-CTA (rank 0)
+        }
+      }
+      __syncwarp();
+    } else {
+      // ---------- O-CTA correction + epilogue (warps 17..20, thread = head) ----------
+      const float* alpha_s = reinterpret_cast<const float*>(base + Smem::kAlpha);
+      const volatile uint32_t* flags = reinterpret_cast<const volatile uint32_t*>(base + Smem::kFlags);
+      const volatile float* stats = reinterpret_cast<const volatile float*>(base + Smem::kStats);
+      bool ok = true;
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const int pb = i & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait_cluster(&bar[B_PFULL + pb], (i >> 1) & 1, p.status, kDevErrTimeout));
+        if (!ok) break;
+        if (flags[pb * 4 + quad] != 0u) {
+          // P(i) was written after MMA2(i-2) completed, so B_ODONE is at most one phase behind:
+          // the parity wait below really waits for MMA2(i-1).
+          ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_ODONE], (i - 1) & 1, p.status, kDevErrTimeout));
+          if (!ok) break;
+          tc_fence_after();
+          const float a = alpha_s[pb * 128 + h];
+#pragma unroll 1
+          for (int c = 0; c < 16; ++c) {
+            uint32_t o[32];
+            tmem_ld32_sync(tmem + lane_base + kColO + 32 * c, o);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * a);
+            tmem_st32(tmem + lane_base + kColO + 32 * c, o);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[B_OREADY + pb]);
+      }
+      ok = __all_sync(0xffffffffu, ok);
+      // B_OFINAL, not B_ODONE: here the per-tile barrier may still be two phases behind, and a
+      // parity wait cannot tell phase ntiles-1 from ntiles-3.
+      if (ok && ntiles > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_OFINAL], 0, p.status, kDevErrTimeout));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_cluster(&bar[B_STATS], 0, p.status, kDevErrTimeout));
+      tc_fence_after();
+      const float m_ref = stats[h], l = stats[128 + h], lr = stats[256 + h];
+      const bool have_o = ok && ntiles > 0;
+      const float inv = (have_o && lr > 0.f) ? 1.f / lr : 0.f;
+      const float lse_nat = (have_o && l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      if (p.nsplit == 1) {
+        uint16_t* dst = p.out + (static_cast<int64_t>(t) * H + h) * kDV;
+#pragma unroll 1
+        for (int c = 0; c < 16; ++c) {
+          uint32_t o[32];
+          if (have_o) {
+            tmem_ld32_sync(tmem + lane_base + kColO + 32 * c, o);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = 0u;
+          }
+          if (h < H) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(o[8 * j + 0]) * inv, __uint_as_float(o[8 * j + 1]) * inv);
+              w.y = pack_bf16x2(__uint_as_float(o[8 * j + 2]) * inv, __uint_as_float(o[8 * j + 3]) * inv);
+              w.z = pack_bf16x2(__uint_as_float(o[8 * j + 4]) * inv, __uint_as_float(o[8 * j + 5]) * inv);
+              w.w = pack_bf16x2(__uint_as_float(o[8 * j + 6]) * inv, __uint_as_float(o[8 * j + 7]) * inv);
+              d4[j] = w;
             }
           }
-          mma_commit(&s_full[sb]);
         }
-        if (it >= 1) {
-          const int i = it - 1, pb = i & 1, s = i % kStages;
-          ok = mbar_wait(&p_full[pb], (i >> 1) & 1, p.status, kDevErrTimeout);
-          if (!ok) break;
-          tc_fence_after();
-          const uint64_t vd = v_desc0 + static_cast<uint64_t>((s * kStageBytes) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < kTileKeys / 16; ++kk) {
-            mma_bf16_ts(tmem + kColO, tmem + kColP + 16 * pb + 8 * kk, vd + static_cast<uint64_t>((kk * 2048) >> 4),
-                        idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(&p_free[pb]);
-          mma_commit(&kv_empty[s]);
-          if (i == ntiles - 1) mma_commit(o_full);
-        }
-      }
-    }
-    __syncwarp();
-  } else {
-    // ---------------- softmax + epilogue (warps 2..5, one head per thread) ----------------
-    // l: sum of the fp32 weights (for the log-sum-exp); lr: sum of the bf16-rounded weights the
-    // P x V MMA actually uses (normalises O, so the output weights sum to one).
-    float m_ref = -INFINITY, l = 0.f, lr = 0.f;
-    bool ok = true;
-    for (int it = 0; it < ntiles && ok; ++it) {
-      const int sb = it & 1;
-      ok = mbar_wait(&s_full[sb], (it >> 1) & 1, p.status, kDevErrTimeout);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      uint32_t sv[32];
-      tmem_ld32(tmem + lane_base + kColS + 32 * sb, sv);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[sb]);
-      float x[32];
-      float tmax = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const int e = it * kTileKeys + c;
-        const bool valid = e < nkeys && rows[e] >= 0;
-        x[c] = valid ? __uint_as_float(sv[c]) * p.scale_log2 : -INFINITY;
-        tmax = fmaxf(tmax, x[c]);
-      }
-      // Lazy rescale, decided per head but executed by the whole warp (TMEM loads/stores are
-      // warp-collective): lanes that keep their reference use alpha = 1.
-      const bool need = tmax > m_ref + kRescaleThreshold;
-      const float alpha = need ? exp2f(m_ref - tmax) : 1.f;  // 0 when m_ref is -inf
-      if (__any_sync(0xffffffffu, need && it >= 1 && m_ref > -INFINITY)) {
-        ok = mbar_wait(&p_free[(it - 1) & 1], ((it - 1) >> 1) & 1, p.status, kDevErrTimeout);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        tc_fence_after();
+        if (h < H && p.lse) p.lse[static_cast<int64_t>(t) * H + h] = lse_nat;
+      } else {
+        const int64_t prow = (static_cast<int64_t>(t) * p.nsplit + split) * H + h;
+        float* dst = p.part_o + prow * kDV;
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 16; ++c) {
           uint32_t o[32];
-          tmem_ld32(tmem + lane_base + kColO + 32 * c, o);
-          tmem_wait_ld();
+          if (have_o) {
+            tmem_ld32_sync(tmem + lane_base + kColO + 32 * c, o);
+          } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tmem + lane_base + kColO + 32 * c, o);
-        }
-        tmem_wait_st();
-      }
-      if (need) {
-        l *= alpha;
-        lr *= alpha;
-        m_ref = tmax;
-      }
-      if (it >= 2) {
-        ok = mbar_wait(&p_free[sb], ((it - 2) >> 1) & 1, p.status, kDevErrTimeout);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        tc_fence_after();
-      }
-      uint32_t pk[16];
+            for (int j = 0; j < 32; ++j) o[j] = 0u;
+          }
+          if (h < H) {
+            float4* d4 = reinterpret_cast<float4*>(dst + 32 * c);
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float p0 = (m_ref > -INFINITY) ? exp2f(x[2 * c] - m_ref) : 0.f;
-        const float p1 = (m_ref > -INFINITY) ? exp2f(x[2 * c + 1] - m_ref) : 0.f;
-        const __nv_bfloat162 bp = __floats2bfloat162_rn(p0, p1);
-        l += p0 + p1;
-        lr += __low2float(bp) + __high2float(bp);
-        pk[c] = *reinterpret_cast<const uint32_t*>(&bp);
-      }
-      tmem_st16(tmem + lane_base + kColP + 16 * sb, pk);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[sb]);
-    }
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok && ntiles > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(o_full, 0, p.status, kDevErrTimeout));
-      tc_fence_after();
-    }
-    const float inv = (lr > 0.f) ? 1.f / lr : 0.f;
-    const float lse_nat = (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
-    const bool have_o = ok && ntiles > 0;
-    if (p.nsplit == 1) {
-      uint16_t* dst = p.out + (static_cast<int64_t>(t) * H + h) * kDV + v * 256;
-#pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        uint32_t o[32];
-        if (have_o) {
-          tmem_ld32(tmem + lane_base + kColO + 32 * c, o);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0u;
-        }
-        if (h < H) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(o[8 * i + 0]) * inv, __uint_as_float(o[8 * i + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv);
-            d4[i] = w;
+            for (int j = 0; j < 8; ++j)
+              d4[j] = make_float4(__uint_as_float(o[4 * j]) * inv, __uint_as_float(o[4 * j + 1]) * inv,
+                                  __uint_as_float(o[4 * j + 2]) * inv, __uint_as_float(o[4 * j + 3]) * inv);
           }
         }
+        if (h < H) p.part_lse[prow] = lse_nat;
       }
-      if (v == 0 && h < H && p.lse) p.lse[static_cast<int64_t>(t) * H + h] = lse_nat;
-    } else {
-      const int64_t prow = (static_cast<int64_t>(t) * p.nsplit + split) * H + h;
-      float* dst = p.part_o + prow * kDV + v * 256;
-#pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        uint32_t o[32];
-        if (have_o) {
-          tmem_ld32(tmem + lane_base + kColO + 32 * c, o);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0u;
-        }
-        if (h < H) {
-          float4* d4 = reinterpret_cast<float4*>(dst + 32 * c);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            d4[i] = make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
-                                __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
-        }
-      }
-      if (v == 0 && h < H) p.part_lse[prow] = lse_nat;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  cluster_sync_all();  // neither CTA leaves while the peer may still touch its shared memory
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -449,10 +613,10 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const float* __restric
 
 int sparse_mla_splits(int T, int k) {
   const int min_splits = (k + kMaxKeysPerCta - 1) / kMaxKeysPerCta;
-  const int ctas = 2 * T;
+  const int clusters_per_wave = 74;  // 148 SMs, two per cluster
   int n = 1;
-  if (ctas > 0 && ctas < 111) n = (148 + ctas - 1) / ctas;
-  const int max_by_tiles = (k + kTileKeys - 1) / kTileKeys;
+  if (T > 0 && T < (3 * clusters_per_wave) / 4) n = (clusters_per_wave + T - 1) / T;
+  const int max_by_tiles = (k + kTile - 1) / kTile;
   if (n > 16) n = 16;
   if (n > max_by_tiles) n = max_by_tiles;
   if (n < min_splits) n = min_splits;
@@ -475,13 +639,13 @@ int launch_sparse_mla(const BatchDev& b, const void* plan, const void* q, int H,
   prm.row_req = pv.row_req;
   prm.row_pos = pv.row_pos;
   prm.q = static_cast<const uint16_t*>(q);
-  prm.kv = static_cast<const uint16_t*>(kv_cache);
+  prm.kv = static_cast<const uint8_t*>(kv_cache);
   prm.S = S;
   prm.k = k;
   prm.H = H;
   prm.nsplit = sparse_mla_splits(b.T, k);
   const int per = (k + prm.nsplit - 1) / prm.nsplit;
-  prm.chunk = (per + kTileKeys - 1) / kTileKeys * kTileKeys;
+  prm.chunk = (per + kTile - 1) / kTile * kTile;
   prm.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634);
   prm.out = static_cast<uint16_t*>(out);
   prm.lse = lse;
@@ -492,18 +656,15 @@ int launch_sparse_mla(const BatchDev& b, const void* plan, const void* q, int H,
   }
   prm.status = &pv.hdr->status;
 
-  CUtensorMap qmap, kvmap;
+  CUtensorMap qmap;
   int e = make_tmap_2d(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, kDLat, static_cast<uint64_t>(b.T) * H,
                        kDLat * 2, 64, 128);
   if (e) return e;
-  e = make_tmap_2d(&kvmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kv_cache, kDLat,
-                   static_cast<uint64_t>(b.num_pages) * kPage, kDLat * 2, 64, 1);
-  if (e) return e;
   cudaError_t ce =
-      cudaFuncSetAttribute(sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, MlaSmem::kDynamic);
+      cudaFuncSetAttribute(sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem::kDynamic);
   if (ce != cudaSuccess) return static_cast<int>(ce);
-  dim3 grid(b.T, 2, prm.nsplit);
-  sparse_mla_kernel<<<grid, kThreads, MlaSmem::kDynamic, static_cast<cudaStream_t>(stream)>>>(qmap, kvmap, prm);
+  dim3 grid(2 * b.T * prm.nsplit, 1, 1);
+  sparse_mla_kernel<<<grid, kThreads, Smem::kDynamic, static_cast<cudaStream_t>(stream)>>>(qmap, prm);
   ce = cudaGetLastError();
   if (ce != cudaSuccess) return static_cast<int>(ce);
   if (prm.nsplit > 1) {
