@@ -56,12 +56,16 @@ constexpr int kMaxTiles = kMaxKeysPerCta / kTile;
 constexpr int kBlk = kTile * 128;            // 128 keys x 64 dims bf16 = 16 KB
 constexpr int kKSlots = 12;                  // S-CTA ring slots (one 64-dim block of one tile each)
 constexpr int kVSlots = 4;                   // O-CTA ring slots (two 64-dim blocks of one tile each)
-constexpr int kProdWarps = 16;               // warps 0..15: gather producers
-constexpr int kGroupWarps = 4;               // warps per producer group (one ring unit per group)
-constexpr int kGroups = kProdWarps / kGroupWarps;
-constexpr int kMmaWarp = kProdWarps;         // warp 16: TMEM allocator and MMA issuer
-constexpr int kSoftWarp0 = kProdWarps + 1;   // warps 17..20: softmax (S-CTA) / correction (O-CTA)
-constexpr int kThreads = 32 * (kProdWarps + 5);
+constexpr int kProdWarps = 12;               // warps 0..11: gather producers
+// A producer group fills one ring unit at a time; each ring slot belongs to exactly one group
+// (slot % groups == group), so a group never runs two uses ahead of the consumer on a slot's
+// barrier, which a parity wait could not tell from one use ahead.
+constexpr int kSGroupWarps = 2, kSGroups = kProdWarps / kSGroupWarps;  // S-CTA: 6 groups, 12 slots
+constexpr int kOGroupWarps = 3, kOGroups = kProdWarps / kOGroupWarps;  // O-CTA: 4 groups, 4 slots
+constexpr int kMmaWarp = kProdWarps;         // warp 12: TMEM allocator and MMA issuer
+constexpr int kSoftWarp0 = kProdWarps + 1;   // warps 13..28: softmax (S-CTA) / correction (O-CTA),
+constexpr int kSoftWarps = 16;               //   four per TMEM lane quadrant, 32 keys / 128 dims each
+constexpr int kThreads = 32 * (kProdWarps + 1 + kSoftWarps);
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
 
 // TMEM columns
@@ -73,7 +77,9 @@ struct Smem {
   // S-CTA
   static constexpr int kQRope = 0;                               // 16 KB
   static constexpr int kKRing = kQRope + kBlk;                   // 12 x 16 KB
-  static constexpr int kSEnd = kKRing + kKSlots * kBlk;          // 208 KB
+  static constexpr int kRed = kKRing + kKSlots * kBlk;           // float [2][4][128]: partial tile max
+  static constexpr int kRedL = kRed + 2 * 4 * 128 * 4;           // float [2][4][128]: partial l, lr
+  static constexpr int kSEnd = kRedL + 2 * 4 * 128 * 4;          // 216 KB
   // O-CTA
   static constexpr int kP = 0;                                   // 2 x 32 KB
   static constexpr int kVRing = kP + 2 * 2 * kBlk;               // 4 x 32 KB
@@ -92,6 +98,8 @@ struct Smem {
   static constexpr int kDynamic = kTotal + 1024;
 };
 static_assert(Smem::kDynamic <= 232448, "sparse MLA shared memory exceeds the 227 KB limit");
+static_assert(kKSlots % kSGroups == 0 && kVSlots % kOGroups == 0, "every ring slot needs a single owner group");
+static_assert(kTile % (4 * kSGroupWarps) == 0, "S-CTA rows per warp");
 
 // barrier indices (same offsets in both CTAs; each CTA initialises the ones it owns)
 enum : int {
@@ -102,9 +110,11 @@ enum : int {
   B_SFULL = B_QROPE + 1,            // [2]  MMA -> softmax
   B_SFREE = B_SFULL + 2,            // [2]  softmax -> MMA (4 warps)
   B_PFREE = B_SFREE + 2,            // [2]  O-CTA MMA -> S-CTA softmax (multicast commit)
-  B_QCONS = B_PFREE + 2,            // 1    softmax warps have moved Q out of the ring (4 warps)
+  B_QCONS = B_PFREE + 2,            // 1    softmax warps have moved Q out of the ring (16 warps)
+  B_QRED = B_QCONS + 1,             // [2][4] partial maxima of one quadrant written (4 warps)
+  B_QEND = B_QRED + 8,              // [4]  partial sums of one quadrant written (4 warps)
   // O-CTA
-  B_VFULL = B_QCONS + 1,            // [4]
+  B_VFULL = B_QEND + 4,             // [4]
   B_VEMPTY = B_VFULL + kVSlots,     // [4]
   B_PFULL = B_VEMPTY + kVSlots,     // [2]  S-CTA softmax -> O-CTA (128 remote arrivals)
   B_OREADY = B_PFULL + 2,           // [2]  correction warps -> MMA (4 warps)
@@ -159,24 +169,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     if (is_s) {
       for (int i = 0; i < kKSlots; ++i) {
-        mbar_init(&bar[B_KFULL + i], 32 * kGroupWarps);  // one cp.async arrival per producer lane
+        mbar_init(&bar[B_KFULL + i], 32 * kSGroupWarps);  // one cp.async arrival per producer lane
         mbar_init(&bar[B_KEMPTY + i], 1);
       }
       mbar_init(&bar[B_QROPE], 1);
-      mbar_init(&bar[B_QCONS], 4);
+      mbar_init(&bar[B_QCONS], kSoftWarps);
+      for (int i = 0; i < 8; ++i) mbar_init(&bar[B_QRED + i], 4);
+      for (int i = 0; i < 4; ++i) mbar_init(&bar[B_QEND + i], 4);
       for (int i = 0; i < 2; ++i) {
         mbar_init(&bar[B_SFULL + i], 1);
-        mbar_init(&bar[B_SFREE + i], 4);
+        mbar_init(&bar[B_SFREE + i], kSoftWarps);
         mbar_init(&bar[B_PFREE + i], 1);
       }
     } else {
       for (int i = 0; i < kVSlots; ++i) {
-        mbar_init(&bar[B_VFULL + i], 32 * kGroupWarps);
+        mbar_init(&bar[B_VFULL + i], 32 * kOGroupWarps);
         mbar_init(&bar[B_VEMPTY + i], 1);
       }
       for (int i = 0; i < 2; ++i) {
-        mbar_init(&bar[B_PFULL + i], 128);
-        mbar_init(&bar[B_OREADY + i], 4);
+        mbar_init(&bar[B_PFULL + i], kSoftWarps);
+        mbar_init(&bar[B_OREADY + i], kSoftWarps);
       }
       mbar_init(&bar[B_ODONE], 1);
       mbar_init(&bar[B_OFINAL], 1);
@@ -216,6 +228,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int quad = warp & 3;
+  const int sub = (warp - kSoftWarp0) >> 2;  // softmax / correction warps: which quarter of the columns
   const int h = quad * 32 + lane;
   const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
 
@@ -243,20 +256,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (warp < kProdWarps) {
       // ---------- S-CTA producers: group g fills units g, g+4, ... (128 keys x 64 dims each) ----------
       // lane l of warp w of the group copies 16-byte chunk (l & 7) of rows 4j + (l >> 3) + 32 w'
-      const int g = warp / kGroupWarps, wg = warp % kGroupWarps;
+      const int g = warp / kSGroupWarps, wg = warp % kSGroupWarps;
       bool ok = ntiles == 0 || mbar_wait(&bar[B_QCONS], 0, p.status, kDevErrTimeout);
       const kv_t* kv = p.kv;
-      for (int u = g; u < ntiles * 9 && ok; u += kGroups) {
+      for (int u = g; u < ntiles * 9 && ok; u += kSGroups) {
         const int i = u / 9, blk = u % 9, slot = u % kKSlots;
         ok = mbar_wait(&bar[B_KEMPTY + slot], ((u / kKSlots) & 1) ^ 1, p.status, kDevErrTimeout);
         if (!ok) break;
         const uint32_t sbase = smem_u32(base + Smem::kKRing + slot * kBlk);
         const int c = lane & 7;
 #pragma unroll 4
-        for (int j = 0; j < kTile / (4 * kGroupWarps); ++j) {
-          const int r = (wg * (kTile / kGroupWarps)) + 4 * j + (lane >> 3);
+        for (int j = 0; j < kTile / (4 * kSGroupWarps); ++j) {
+          const int r = (wg * (kTile / kSGroupWarps)) + 4 * j + (lane >> 3);
           const int prow = max(rows[i * kTile + r], 0);
-          cp_async_16(sbase + r * 128 + (((c ^ (r & 7))) << 4), kv + static_cast<int64_t>(prow) * kRowBytes + blk * 128 + c * 16);
+          cp_async_16(sbase + r * 128 + ((c ^ (r & 7)) << 4), kv + static_cast<int64_t>(prow) * kRowBytes + blk * 128 + c * 16);
         }
         cp_async_mbar_arrive_noinc(&bar[B_KFULL + slot]);
       }
@@ -299,20 +312,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     } else {
-      // ---------- S-CTA softmax (warps 17..20, thread = head) ----------
+      // ---------- S-CTA softmax (warps 15..30: thread = head h, keys 32*sub .. 32*sub+31) ----------
       const uint32_t peer_p = peer_addr(smem_u32(base + Smem::kP), 1);
       const uint32_t peer_alpha = peer_addr(smem_u32(base + Smem::kAlpha), 1);
       const uint32_t peer_flags = peer_addr(smem_u32(base + Smem::kFlags), 1);
       const uint32_t peer_stats = peer_addr(smem_u32(base + Smem::kStats), 1);
       const uint32_t peer_pfull = peer_addr(smem_u32(&bar[B_PFULL]), 1);
       const uint32_t peer_statbar = peer_addr(smem_u32(&bar[B_STATS]), 1);
+      float* red = reinterpret_cast<float*>(base + Smem::kRed);    // [2][4][128]
+      float* redl = reinterpret_cast<float*>(base + Smem::kRedL);  // [2][4][128]: l, lr
       float m_ref = -INFINITY, l = 0.f, lr = 0.f;
       bool ok = true;
       if (ntiles > 0) {
-        // Q dims 0..511: 8 swizzled blocks in ring slots 0..7 -> TMEM columns 256..511 (lane = head)
+        // Q dims 0..511: swizzled blocks 2*sub, 2*sub+1 of ring slots 0..7 -> TMEM (lane = head)
         ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_QROPE], 0, p.status, kDevErrTimeout));
         if (ok) {
-          for (int blk = 0; blk < 8; ++blk) {
+          for (int blk = 2 * sub; blk < 2 * sub + 2; ++blk) {
             const uint8_t* rowp = base + Smem::kKRing + blk * kBlk + h * 128;
             uint32_t r[32];
 #pragma unroll
@@ -336,18 +351,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_SFULL + sb], (i >> 1) & 1, p.status, kDevErrTimeout));
         if (!ok) break;
         tc_fence_after();
-        const uint32_t srow = tmem + lane_base + kColS + kTile * sb;
-        // pass 1: tile maximum (scaled, log2 units) over the valid keys
-        float tmax = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          tmem_ld32_sync(srow + 32 * c, v);
-          const uint32_t m = masks[4 * i + c];
+        uint32_t v[32];
+        tmem_ld32_sync(tmem + lane_base + kColS + kTile * sb + 32 * sub, v);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[B_SFREE + sb]);
+        const uint32_t m = masks[4 * i + sub];
+        float pmax = -INFINITY;
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if ((m >> j) & 1u) tmax = fmaxf(tmax, __uint_as_float(v[j]) * p.scale_log2);
-        }
+        for (int j = 0; j < 32; ++j)
+          if ((m >> j) & 1u) pmax = fmaxf(pmax, __uint_as_float(v[j]) * p.scale_log2);
+        // tile maximum of head h across the four warps of this quadrant (shared memory + mbarrier)
+        red[(sb * 4 + sub) * 128 + h] = pmax;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[B_QRED + sb * 4 + quad]);
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_QRED + sb * 4 + quad], (i >> 1) & 1, p.status, kDevErrTimeout));
+        if (!ok) break;
+        const float tmax = fmaxf(fmaxf(red[(sb * 4 + 0) * 128 + h], red[(sb * 4 + 1) * 128 + h]),
+                                 fmaxf(red[(sb * 4 + 2) * 128 + h], red[(sb * 4 + 3) * 128 + h]));
         const bool need = tmax > m_ref + kRescaleThreshold;
         const float alpha = need ? exp2f(m_ref - tmax) : 1.f;  // 0 when m_ref is -inf
         if (need) {
@@ -359,46 +380,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // the O-CTA must be done with the P buffer of tile i-2
         ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_PFREE + sb], ((i >> 1) & 1) ^ 1, p.status, kDevErrTimeout));
         if (!ok) break;
-        // pass 2: P row h (128 keys, bf16) into the peer's K-major swizzled buffer (2 blocks of 64)
+        // P[h, 32*sub .. +31] (bf16) into the peer's K-major swizzled buffer (2 blocks of 64 keys)
+        const float m_use = (m_ref > -INFINITY) ? m_ref : 0.f;  // m_ref = -inf: every key so far masked
         const uint32_t prow = peer_p + static_cast<uint32_t>(sb * 2 * kBlk + h * 128);
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          tmem_ld32_sync(srow + 32 * c, v);
-          const uint32_t m = masks[4 * i + c];
 #pragma unroll
-          for (int q8 = 0; q8 < 4; ++q8) {  // 8 keys = one 16-byte chunk
-            uint32_t w[4];
+        for (int q8 = 0; q8 < 4; ++q8) {  // 8 keys = one 16-byte chunk
+          uint32_t w[4];
 #pragma unroll
-            for (int q2 = 0; q2 < 4; ++q2) {
-              const int j0 = 8 * q8 + 2 * q2;
-              const float p0 = ((m >> j0) & 1u) && m_ref > -INFINITY
-                                   ? exp2f(__uint_as_float(v[j0]) * p.scale_log2 - m_ref) : 0.f;
-              const float p1 = ((m >> (j0 + 1)) & 1u) && m_ref > -INFINITY
-                                   ? exp2f(__uint_as_float(v[j0 + 1]) * p.scale_log2 - m_ref) : 0.f;
-              const __nv_bfloat162 bp = __floats2bfloat162_rn(p0, p1);
-              l += p0 + p1;
-              lr += __low2float(bp) + __high2float(bp);
-              w[q2] = *reinterpret_cast<const uint32_t*>(&bp);
-            }
-            const int chunk = 4 * c + q8;  // 0..15: block chunk>>3, chunk-in-block chunk&7
-            const uint32_t addr = prow + static_cast<uint32_t>((chunk >> 3) * kBlk + (((chunk & 7) ^ (h & 7)) << 4));
-            st_cluster_v4(addr, w[0], w[1], w[2], w[3]);
+          for (int q2 = 0; q2 < 4; ++q2) {
+            const int j0 = 8 * q8 + 2 * q2;
+            const float p0 = ((m >> j0) & 1u) ? fast_exp2(fmaf(__uint_as_float(v[j0]), p.scale_log2, -m_use)) : 0.f;
+            const float p1 = ((m >> (j0 + 1)) & 1u) ? fast_exp2(fmaf(__uint_as_float(v[j0 + 1]), p.scale_log2, -m_use)) : 0.f;
+            const __nv_bfloat162 bp = __floats2bfloat162_rn(p0, p1);
+            l += p0 + p1;
+            lr += __low2float(bp) + __high2float(bp);
+            w[q2] = *reinterpret_cast<const uint32_t*>(&bp);
+          }
+          const int chunk = 4 * sub + q8;  // 0..15: block chunk>>3, chunk-in-block chunk&7
+          st_cluster_v4(prow + static_cast<uint32_t>((chunk >> 3) * kBlk + (((chunk & 7) ^ (h & 7)) << 4)), w[0], w[1],
+                        w[2], w[3]);
+        }
+        if (sub == 0) {
+          st_cluster_f32(peer_alpha + static_cast<uint32_t>((sb * 128 + h) * 4), alpha);
+          if (lane == 0) st_cluster_u32(peer_flags + static_cast<uint32_t>((sb * 4 + quad) * 4), warp_rescale ? 1u : 0u);
+        }
+        fence_proxy_async_cluster();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(peer_pfull + static_cast<uint32_t>(sb * 8));
+      }
+      // per-head sums over the four warps of the quadrant, then the final statistics (always sent,
+      // so the O-CTA never waits in vain)
+      redl[(0 * 4 + sub) * 128 + h] = l;
+      redl[(1 * 4 + sub) * 128 + h] = lr;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[B_QEND + quad]);
+      const bool sums_ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_QEND + quad], 0, p.status, kDevErrTimeout));
+      if (sub == 0) {
+        float lt = 0.f, lrt = 0.f;
+        if (sums_ok) {
+          for (int q = 0; q < 4; ++q) {
+            lt += redl[(0 * 4 + q) * 128 + h];
+            lrt += redl[(1 * 4 + q) * 128 + h];
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[B_SFREE + sb]);
-        st_cluster_f32(peer_alpha + static_cast<uint32_t>((sb * 128 + h) * 4), alpha);
-        if (lane == 0) st_cluster_u32(peer_flags + static_cast<uint32_t>((sb * 4 + quad) * 4), warp_rescale ? 1u : 0u);
-        fence_proxy_async_cluster();
-        mbar_arrive_remote(peer_pfull + static_cast<uint32_t>(sb * 8));
+        st_cluster_f32(peer_stats + static_cast<uint32_t>(h * 4), m_ref);
+        st_cluster_f32(peer_stats + static_cast<uint32_t>((128 + h) * 4), lt);
+        st_cluster_f32(peer_stats + static_cast<uint32_t>((256 + h) * 4), lrt);
+        mbar_arrive_remote(peer_statbar);
       }
-      // final statistics for the epilogue, always sent so the O-CTA never waits in vain
-      st_cluster_f32(peer_stats + static_cast<uint32_t>(h * 4), m_ref);
-      st_cluster_f32(peer_stats + static_cast<uint32_t>((128 + h) * 4), l);
-      st_cluster_f32(peer_stats + static_cast<uint32_t>((256 + h) * 4), lr);
-      mbar_arrive_remote(peer_statbar);
       // the last multicast commits of the O-CTA land in this CTA's barriers: wait for them
       if (ok && ntiles > 0) {
         const int i1 = ntiles - 1;
@@ -410,18 +439,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (warp < kProdWarps) {
       // ---------- O-CTA producers: V in units of 128 keys x 128 dims (2 blocks), one unit per group ----
       // lane l copies 16-byte chunk (l & 15) of rows 2j + (l >> 4) of its warp's quarter of the unit
-      const int g = warp / kGroupWarps, wg = warp % kGroupWarps;
+      const int g = warp / kOGroupWarps, wg = warp % kOGroupWarps;
+      const int r_lo = (wg * kTile) / kOGroupWarps, r_hi = ((wg + 1) * kTile) / kOGroupWarps;
       const kv_t* kv = p.kv;
       bool ok = true;
-      for (int u = g; u < ntiles * 4 && ok; u += kGroups) {
+      for (int u = g; u < ntiles * 4 && ok; u += kOGroups) {
         const int i = u / 4, qd = u % 4, slot = u % kVSlots;
         ok = mbar_wait(&bar[B_VEMPTY + slot], ((u / kVSlots) & 1) ^ 1, p.status, kDevErrTimeout);
         if (!ok) break;
         const uint32_t sbase = smem_u32(base + Smem::kVRing + slot * 2 * kBlk);
         const int c = lane & 15;
 #pragma unroll 4
-        for (int j = 0; j < kTile / (2 * kGroupWarps); ++j) {
-          const int r = (wg * (kTile / kGroupWarps)) + 2 * j + (lane >> 4);
+        for (int r = r_lo + (lane >> 4); r < r_hi; r += 2) {  // 16 lanes per 256-byte row segment
           const int prow = max(rows[i * kTile + r], 0);
           cp_async_16(sbase + (c >> 3) * kBlk + r * 128 + (((c & 7) ^ (r & 7)) << 4),
                       kv + static_cast<int64_t>(prow) * kRowBytes + qd * 256 + c * 16);
@@ -466,10 +495,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     } else {
-      // ---------- O-CTA correction + epilogue (warps 17..20, thread = head) ----------
+      // ---------- O-CTA correction + epilogue (warps 15..30: head h, O columns 128*sub .. +127) -------
       const float* alpha_s = reinterpret_cast<const float*>(base + Smem::kAlpha);
       const volatile uint32_t* flags = reinterpret_cast<const volatile uint32_t*>(base + Smem::kFlags);
       const volatile float* stats = reinterpret_cast<const volatile float*>(base + Smem::kStats);
+      const uint32_t ocol = tmem + lane_base + kColO + 128 * sub;
       bool ok = true;
       for (int i = 0; i < ntiles && ok; ++i) {
         const int pb = i & 1;
@@ -483,12 +513,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const float a = alpha_s[pb * 128 + h];
 #pragma unroll 1
-          for (int c = 0; c < 16; ++c) {
+          for (int c = 0; c < 4; ++c) {
             uint32_t o[32];
-            tmem_ld32_sync(tmem + lane_base + kColO + 32 * c, o);
+            tmem_ld32_sync(ocol + 32 * c, o);
 #pragma unroll
             for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * a);
-            tmem_st32(tmem + lane_base + kColO + 32 * c, o);
+            tmem_st32(ocol + 32 * c, o);
           }
           tmem_wait_st();
           tc_fence_before();
@@ -507,12 +537,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const float inv = (have_o && lr > 0.f) ? 1.f / lr : 0.f;
       const float lse_nat = (have_o && l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
       if (p.nsplit == 1) {
-        uint16_t* dst = p.out + (static_cast<int64_t>(t) * H + h) * kDV;
+        uint16_t* dst = p.out + (static_cast<int64_t>(t) * H + h) * kDV + 128 * sub;
 #pragma unroll 1
-        for (int c = 0; c < 16; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
           if (have_o) {
-            tmem_ld32_sync(tmem + lane_base + kColO + 32 * c, o);
+            tmem_ld32_sync(ocol + 32 * c, o);
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j) o[j] = 0u;
@@ -530,15 +560,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (h < H && p.lse) p.lse[static_cast<int64_t>(t) * H + h] = lse_nat;
+        if (sub == 0 && h < H && p.lse) p.lse[static_cast<int64_t>(t) * H + h] = lse_nat;
       } else {
         const int64_t prow = (static_cast<int64_t>(t) * p.nsplit + split) * H + h;
-        float* dst = p.part_o + prow * kDV;
+        float* dst = p.part_o + prow * kDV + 128 * sub;
 #pragma unroll 1
-        for (int c = 0; c < 16; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
           if (have_o) {
-            tmem_ld32_sync(tmem + lane_base + kColO + 32 * c, o);
+            tmem_ld32_sync(ocol + 32 * c, o);
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j) o[j] = 0u;
@@ -551,7 +581,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                   __uint_as_float(o[4 * j + 2]) * inv, __uint_as_float(o[4 * j + 3]) * inv);
           }
         }
-        if (h < H) p.part_lse[prow] = lse_nat;
+        if (sub == 0 && h < H) p.part_lse[prow] = lse_nat;
       }
     }
   }
