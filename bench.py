@@ -82,6 +82,29 @@ def _positions(hb):
 
 
 # ---------------------------------------------------------------------------------------------
+# multi-rank plumbing: every rank runs its own batch (weak scaling by request), no data exchange
+
+def rank_seed(rank: int) -> int:
+    """Seed of the synthetic batch a rank runs: ranks own disjoint, equally shaped batches."""
+    return rank
+
+
+def max_over_ranks(value: float, dist=None, device="cpu") -> float:
+    """The largest per-rank value (timings are reported as the slowest rank's)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(rows_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job query tokens per second: all ranks' rows over the slowest rank's step time."""
+    return world * rows_per_rank / (ms / 1e3)
+
+
+# ---------------------------------------------------------------------------------------------
 # clocks sampled during the timed region
 
 class ClockSampler:
@@ -237,7 +260,7 @@ def main():
     torch.cuda.set_device(dev)
     dsa.load()
 
-    hb = synth.make_batch(wl, seed=rank)
+    hb = synth.make_batch(wl, seed=rank_seed(rank))
     db = dsa.DeviceBatch(hb, device=dev)
     T = hb.total_q
     stream = torch.cuda.current_stream()
@@ -274,12 +297,8 @@ def main():
             ends[i].record(stream)
         barrier()
     times = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    ms = statistics.mean(times)
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms = float(ms_t.item())
-    value = world * T / (ms / 1e3)
+    ms = max_over_ranks(statistics.mean(times), dist, dev)
+    value = job_throughput(T, world, ms)
 
     # per-stage timings of the same kernels (roofline of the dominant one)
     plan_t = dsa.plan(db.batch, db.nhI)
@@ -353,12 +372,9 @@ def main():
             es.append(a)
             ee.append(b)
         barrier()
-        e_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(es, ee))
-        e_t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-        if dist is not None:
-            dist.all_reduce(e_t, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * T / (float(e_t.item()) / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "ms_per_step": float(e_t.item())}
+        e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in zip(es, ee)), dist, dev)
+        e2e = {"value": job_throughput(T, world, e_ms), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": e_ms}
 
     if dist is not None:
         dist.barrier()
