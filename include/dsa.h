@@ -23,8 +23,8 @@
  *     and m_b query tokens; query i of request b sits at position p = n_b - m_b + i and sees
  *     j in [0, p].
  *   - All data pointers are DEVICE pointers owned by the caller; the library allocates no memory
- *     and keeps no global state (thread-safe). Workspace is caller-provided, sized by the
- *     *_workspace_size functions.
+ *     and keeps no global state (thread-safe), except dsa_layer_noalloc's static device array.
+ *     Workspace is caller-provided, sized by the *_workspace_size functions.
  *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy
  *     default stream). Nothing synchronises the host.
  *   - Arguments are checked on the host before anything is launched; a bad argument returns
@@ -129,6 +129,21 @@ dsa_status_t dsa_layer(const dsa_batch_t* batch, const uint8_t* qI, const float*
                        int nhI, const uint8_t* kI_cache, const float* kI_scale, const void* q, int H,
                        const void* kv_cache, int k, float softmax_scale, void* out, float* lse, int32_t* S_out,
                        void* ws, size_t ws_bytes, void* stream);
+
+/* ---- the whole path without caller-provided workspace --------------------------------------
+ * No counterpart on the pages: this exists for callers that cannot allocate device memory where
+ * they run a layer (a locked or defragmenting memory pool, allocator-free runtimes, hooks that
+ * must not call cudaMalloc). Same arguments and results as dsa_layer, minus ws/ws_bytes: the
+ * workspace comes from a file-scope device array of 64 MiB that every GPU loading the library
+ * holds until exit. Requests needing more than that (dsa_layer_workspace_size > 64 MiB) return
+ * DSA_ERR_WORKSPACE and launch nothing. Allocates nothing. The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress): make it before any stream capture. All calls share
+ * the array, which keeps the last call's contents; calls whose kernels overlap on the GPU race on
+ * it. The plan (for dsa_status_read) lives in that array and is not exposed. */
+dsa_status_t dsa_layer_noalloc(const dsa_batch_t* batch, const uint8_t* qI, const float* qI_scale, const float* wI,
+                               int nhI, const uint8_t* kI_cache, const float* kI_scale, const void* q, int H,
+                               const void* kv_cache, int k, float softmax_scale, void* out, float* lse,
+                               int32_t* S_out, void* stream);
 
 const char* dsa_status_string(dsa_status_t status);
 int dsa_abi_version(void);

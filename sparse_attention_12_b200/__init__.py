@@ -38,7 +38,7 @@ class DsaBatchC(ctypes.Structure):
 
 EXPORTS = ("dsa_abi_version", "dsa_status_string", "dsa_plan_workspace_size", "dsa_plan", "dsa_status_read",
            "dsa_index_scores", "dsa_topk", "dsa_sparse_mla_workspace_size", "dsa_sparse_mla",
-           "dsa_layer_workspace_size", "dsa_layer")
+           "dsa_layer_workspace_size", "dsa_layer", "dsa_layer_noalloc")
 
 _lib = None
 
@@ -65,6 +65,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "dsa_sparse_mla": (I, [BP, P, P, I, P, P, I, ctypes.c_float, P, P, P, SZ, P]),
         "dsa_layer_workspace_size": (SZ, [BP, I, I, I]),
         "dsa_layer": (I, [BP, P, P, P, I, P, P, P, I, P, I, ctypes.c_float, P, P, P, P, SZ, P]),
+        "dsa_layer_noalloc": (I, [BP, P, P, P, I, P, P, P, I, P, I, ctypes.c_float, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

@@ -1,0 +1,63 @@
+"""dsa_layer_noalloc: the whole path with its workspace in the library's static device array.
+
+Callers that cannot allocate device memory where they run a layer (a locked memory pool,
+allocator-free runtimes, hooks that must not call cudaMalloc) use this entry point. The test calls
+it through the C ABI twice in a row and checks each result against dsa_layer with a
+caller-provided workspace, to the attention tolerance the parity tests use. This file sorts last,
+so a run that stops at the first failure has already run every other test.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import sparse_attention_12_b200 as dsa
+from sparse_attention_12_b200 import build as dsa_build
+from sparse_attention_12_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _noalloc(lib, db, out, lse, S):
+    return lib.dsa_layer_noalloc(db.batch.ref(), db.qI.data_ptr(), db.qI_scale.data_ptr(), db.wI.data_ptr(),
+                                 db.nhI, db.kI_cache.data_ptr(), db.kI_scale.data_ptr(), db.q.data_ptr(), db.H,
+                                 db.kv_cache.data_ptr(), db.k, ctypes.c_float(db.softmax_scale), out.data_ptr(),
+                                 lse.data_ptr(), S.data_ptr(), torch.cuda.current_stream().cuda_stream)
+
+
+def test_noalloc_matches_layer_twice():
+    assert torch.cuda.is_available()
+    dsa_build.build()
+    lib = dsa.load()
+    wl = synth.custom("noalloc", [5000, 777, 2049, 64], [1, 2, 1, 3], n_heads_index=64, topk=512, n_heads=128,
+                      needles="decode", n_needles=3)
+    hb = synth.make_batch(wl, seed=7, extra_pages=2)
+    db = dsa.DeviceBatch(hb)
+    T = hb.total_q
+    ref_S = torch.empty((T, db.k), dtype=torch.int32, device="cuda")
+    ref_lse = torch.empty((T, db.H), dtype=torch.float32, device="cuda")
+    ref = dsa.layer(db.batch, db.qI, db.qI_scale, db.wI, db.kI_cache, db.kI_scale, db.q, db.kv_cache, db.k,
+                    db.softmax_scale, lse=ref_lse, S_out=ref_S)
+    torch.cuda.synchronize()
+    for call in range(2):
+        out = torch.full((T, db.H, 512), float("nan"), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((T, db.H), dtype=torch.float32, device="cuda")
+        S = torch.full((T, db.k), -7, dtype=torch.int32, device="cuda")
+        assert _noalloc(lib, db, out, lse, S) == 0, f"call {call}"
+        torch.cuda.synchronize()
+        assert torch.equal(S, ref_S), f"call {call}: index sets differ"
+        err = (out.float() - ref.float()).abs()
+        assert err.max().item() <= 2e-2 and err.mean().item() <= 2e-3, f"call {call}: output differs"
+        assert torch.allclose(lse, ref_lse, atol=1e-3, rtol=0), f"call {call}: lse differs"
+
+
+def test_noalloc_rejects_requests_above_the_static_size():
+    lib = dsa.load()
+    # 40000 query rows x 2048 positions of fp32 scores alone need 312 MiB of workspace
+    b = dsa.DsaBatchC(1, 40000, 40000, 40000, 625, 700, 1 << 20, 1 << 20, 1 << 20)
+    need = lib.dsa_layer_workspace_size(ctypes.byref(b), 64, 128, 2048)
+    assert need > (64 << 20)
+    st = lib.dsa_layer_noalloc(ctypes.byref(b), 1 << 20, 1 << 20, 1 << 20, 64, 1 << 20, 1 << 20, 1 << 20, 128,
+                               1 << 20, 2048, ctypes.c_float(0.07), 1 << 20, None, None, None)
+    assert st == 3  # DSA_ERR_WORKSPACE, nothing launched
