@@ -39,6 +39,24 @@ DEFAULT_WORKLOAD = "decode_64x16k"
 L2_FLUSH_BYTES = 256 << 20
 
 
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu record, or None when there is no
+    record for this workload or the kernel's source changed since the counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "roofline_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel]
+        if rec["workload"] != workload:
+            return None
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+                return None
+        return int(rec["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -398,7 +416,8 @@ def main():
                    "topk": wl.topk, "index_heads": wl.n_heads_index, "heads": wl.n_heads, "page_size": 64,
                    "l2": "256 MiB flush between timed steps", "parallelism": f"{world} independent ranks"},
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": None, "peak_source": peak_src},
+                     "frac": achieved / hbm_peak, "algorithmic_bytes": dom_bytes,
+                     "traffic": recorded_traffic(dominant + "_kernel", wl.name), "peak_source": peak_src},
         "layer_roofline": {"algorithmic_bytes": total_bytes,
                            "achieved_GBps": total_bytes / (ms / 1e3) / 1e9,
                            "frac": total_bytes / (ms / 1e3) / 1e9 / hbm_peak},
