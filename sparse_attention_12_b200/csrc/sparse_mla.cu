@@ -12,24 +12,25 @@
 //   S-CTA (rank 0): S = Q C^T and the softmax.
 //     * Q (128 heads x 576 bf16): dims 0..511 in TMEM as the A operand (256 columns), the 64 rope
 //       dims in shared memory (one 128-byte-swizzled block).
-//     * The selected latent rows are gathered by 16 producer warps with 16-byte cp.async (8 lanes
-//       per 128-byte row segment, XOR-swizzled on the way into the canonical 128-byte-swizzled
-//       K-major UMMA layout) into a 12-slot ring of 128 keys x 64 dims. Random 1152-byte rows need
-//       hundreds of loads in flight per SM; TMA gather4 tops out near 2 TB/s here (per-copy cost).
+//     * 20 producer warps gather the selected latent rows with 16-byte cp.async (8 lanes per
+//       128-byte row segment, XOR-swizzled on the way into the canonical 128-byte-swizzled K-major
+//       UMMA layout) into a 10-slot ring of 128 keys x 64 dims. Random 1152-byte rows need
+//       hundreds of loads in flight per SM; TMA gather4 tops out near 2 TB/s (per-copy cost).
 //     * Each tile of 128 keys costs 36 tcgen05.mma (M=128 heads, N=128 keys, K=16), which run at
 //       the full bf16 rate; S tiles are double-buffered in TMEM (2 x 128 columns).
-//     * Four softmax warps (thread = head) read each S tile twice from TMEM (maximum, then
-//       exponentials, to keep registers low) and turn it into P (bf16) with an online softmax whose
-//       reference maximum only moves when a tile's maximum exceeds it by more than 2^8, and store
-//       P, the per-head rescale factor and a per-warp "rescale" flag straight into the O-CTA's
-//       shared memory (distributed shared memory), then arrive on the O-CTA's barrier.
+//     * Eight softmax warps (two per TMEM lane quadrant, 64 keys each) read S twice (maximum, then
+//       exponentials), keep an online softmax whose reference maximum only moves when a tile's
+//       maximum exceeds it by more than 2^8, and write bf16 P, the per-head rescale factors and
+//       per-quadrant rescale flags into a local staging buffer; a copier warp ships the 33 KB block
+//       to the O-CTA with a single bulk copy that completes on the O-CTA's barrier.
 //   O-CTA (rank 1): O = P V.
-//     * O (128 heads x 512 fp32) fills its whole TMEM. V = c[0:512] of the same rows is gathered
-//       by its own 16 producer warps in units of 128 keys x 128 dims (4 per tile).
+//     * O (128 heads x 512 fp32) fills its whole TMEM. V = c[0:512] of the same rows (mostly L2
+//       hits: the S-CTA fetched them) is gathered by 20 producer warps in units of 128 keys x 128
+//       dims (4 per tile).
 //     * Per tile: 32 tcgen05.mma (M=128, N=128 dims, K=16 keys), A = P (shared memory, K-major),
 //       B = V (MN-major). Completion is multicast back to the S-CTA to free the P buffer.
-//     * Four correction warps rescale O rows in TMEM when the S-CTA flags a new reference
-//       maximum (rare), and at the end normalise O and write the output.
+//     * Eight correction warps rescale O rows in TMEM when a quadrant is flagged (rare), and at
+//       the end normalise O and write the output.
 //
 // Splits (several clusters over one S_t) write normalised partial outputs and their log-sum-exp
 // to the workspace; a combine kernel merges them: o = sum_s exp(lse_s - lse) o_s.
@@ -48,24 +49,25 @@ int make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, co
 
 namespace {
 
-using kv_t = uint8_t;
 constexpr int kRowBytes = kDLat * 2;         // 1152
 constexpr int kTile = 128;                   // keys per tile (MMA N for S, K-extent for P V)
 constexpr int kMaxKeysPerCta = 2048;         // S_t entries one cluster handles
 constexpr int kMaxTiles = kMaxKeysPerCta / kTile;
 constexpr int kBlk = kTile * 128;            // 128 keys x 64 dims bf16 = 16 KB
-constexpr int kKSlots = 12;                  // S-CTA ring slots (one 64-dim block of one tile each)
+constexpr int kKSlots = 10;                  // S-CTA ring slots (one 64-dim block of one tile each)
 constexpr int kVSlots = 4;                   // O-CTA ring slots (two 64-dim blocks of one tile each)
-constexpr int kProdWarps = 12;               // warps 0..11: gather producers
+constexpr int kProdWarps = 20;               // warps 0..19: gather producers
 // A producer group fills one ring unit at a time; each ring slot belongs to exactly one group
 // (slot % groups == group), so a group never runs two uses ahead of the consumer on a slot's
 // barrier, which a parity wait could not tell from one use ahead.
-constexpr int kSGroupWarps = 2, kSGroups = kProdWarps / kSGroupWarps;  // S-CTA: 6 groups, 12 slots
-constexpr int kOGroupWarps = 3, kOGroups = kProdWarps / kOGroupWarps;  // O-CTA: 4 groups, 4 slots
-constexpr int kMmaWarp = kProdWarps;         // warp 12: TMEM allocator and MMA issuer
-constexpr int kSoftWarp0 = kProdWarps + 1;   // warps 13..28: softmax (S-CTA) / correction (O-CTA),
-constexpr int kSoftWarps = 16;               //   four per TMEM lane quadrant, 32 keys / 128 dims each
-constexpr int kThreads = 32 * (kProdWarps + 1 + kSoftWarps);
+constexpr int kSGroupWarps = 4, kSGroups = kProdWarps / kSGroupWarps;  // S-CTA: 5 groups, 10 slots
+constexpr int kOGroupWarps = 5, kOGroups = kProdWarps / kOGroupWarps;  // O-CTA: 4 groups, 4 slots
+constexpr int kMmaWarp = kProdWarps;         // warp 20: TMEM allocator and MMA issuer
+constexpr int kSoftWarp0 = kProdWarps + 1;   // warps 21..28: softmax (S-CTA) / correction (O-CTA),
+constexpr int kSoftWarps = 8;                //   two per TMEM lane quadrant
+constexpr int kSubs = kSoftWarps / 4;        // column halves per quadrant
+constexpr int kCopyWarp = kSoftWarp0 + kSoftWarps;  // warp 29: ships P blocks (S-CTA only)
+constexpr int kThreads = 32 * (kCopyWarp + 1);
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
 
 // TMEM columns
@@ -73,19 +75,26 @@ constexpr uint32_t kColS = 0;      // S-CTA: S tiles at 0 and 128
 constexpr uint32_t kColQ = 256;    // S-CTA: Q dims 0..511
 constexpr uint32_t kColO = 0;      // O-CTA: O, 512 columns
 
+// A P block as shipped from the S-CTA to the O-CTA: P (two 64-key blocks of [128 heads][128 B],
+// swizzled), alpha[128] floats, flags[4] words.
+constexpr int kPBytes = 2 * kBlk;
+constexpr int kPAlpha = kPBytes;
+constexpr int kPFlags = kPAlpha + 128 * 4;
+constexpr int kPShip = kPFlags + 4 * 4;      // 33296 bytes, a multiple of 16
+constexpr int kPStride = 33 * 1024;          // keeps every P block 1024-byte aligned
+
 struct Smem {
   // S-CTA
   static constexpr int kQRope = 0;                               // 16 KB
-  static constexpr int kKRing = kQRope + kBlk;                   // 12 x 16 KB
-  static constexpr int kRed = kKRing + kKSlots * kBlk;           // float [2][4][128]: partial tile max
-  static constexpr int kRedL = kRed + 2 * 4 * 128 * 4;           // float [2][4][128]: partial l, lr
-  static constexpr int kSEnd = kRedL + 2 * 4 * 128 * 4;          // 216 KB
+  static constexpr int kKRing = kQRope + kBlk;                   // 10 x 16 KB
+  static constexpr int kPStage = kKRing + kKSlots * kBlk;        // one P block being assembled
+  static constexpr int kRed = kPStage + kPStride;                // float [2][kSubs][128]: tile maxima
+  static constexpr int kRedL = kRed + 2 * kSubs * 128 * 4;       // float [2][kSubs][128]: l, lr
+  static constexpr int kSEnd = kRedL + 2 * kSubs * 128 * 4;
   // O-CTA
-  static constexpr int kP = 0;                                   // 2 x 32 KB
-  static constexpr int kVRing = kP + 2 * 2 * kBlk;               // 4 x 32 KB
-  static constexpr int kAlpha = kVRing + kVSlots * 2 * kBlk;     // float [2][128]
-  static constexpr int kFlags = kAlpha + 2 * 128 * 4;            // u32 [2][4]
-  static constexpr int kStats = kFlags + 2 * 4 * 4;              // float [3][128]: m, l, lr
+  static constexpr int kP = 0;                                   // 2 P blocks, kPStride apart
+  static constexpr int kVRing = kP + 2 * kPStride;               // 4 x 32 KB
+  static constexpr int kStats = kVRing + kVSlots * 2 * kBlk;     // float [3][128]: m, l, lr
   static constexpr int kOEnd = kStats + 3 * 128 * 4;
   // both
   static constexpr int kCommon = (kSEnd > kOEnd ? kSEnd : kOEnd);
@@ -98,26 +107,30 @@ struct Smem {
   static constexpr int kDynamic = kTotal + 1024;
 };
 static_assert(Smem::kDynamic <= 232448, "sparse MLA shared memory exceeds the 227 KB limit");
+static_assert(kPShip <= kPStride && kPShip % 16 == 0, "P block");
 static_assert(kKSlots % kSGroups == 0 && kVSlots % kOGroups == 0, "every ring slot needs a single owner group");
 static_assert(kTile % (4 * kSGroupWarps) == 0, "S-CTA rows per warp");
+static_assert(kTile == 32 * 2 * kSubs, "softmax warps cover a tile");
 
 // barrier indices (same offsets in both CTAs; each CTA initialises the ones it owns)
 enum : int {
   // S-CTA
-  B_KFULL = 0,                      // [12]
-  B_KEMPTY = B_KFULL + kKSlots,     // [12]
-  B_QROPE = B_KEMPTY + kKSlots,     // 1
-  B_SFULL = B_QROPE + 1,            // [2]  MMA -> softmax
-  B_SFREE = B_SFULL + 2,            // [2]  softmax -> MMA (4 warps)
-  B_PFREE = B_SFREE + 2,            // [2]  O-CTA MMA -> S-CTA softmax (multicast commit)
-  B_QCONS = B_PFREE + 2,            // 1    softmax warps have moved Q out of the ring (16 warps)
-  B_QRED = B_QCONS + 1,             // [2][4] partial maxima of one quadrant written (4 warps)
-  B_QEND = B_QRED + 8,              // [4]  partial sums of one quadrant written (4 warps)
+  B_KFULL = 0,                      // [10] cp.async arrivals of one producer group
+  B_KEMPTY = B_KFULL + kKSlots,     // [10] MMA commit
+  B_QROPE = B_KEMPTY + kKSlots,     // 1    TMA of Q
+  B_QCONS = B_QROPE + 1,            // 1    softmax warps moved Q out of the ring (8 warps)
+  B_QRED = B_QCONS + 1,             // [2][4] partial maxima of one quadrant written (kSubs warps)
+  B_QEND = B_QRED + 8,              // [4]  partial sums of one quadrant written (kSubs warps)
+  B_SFULL = B_QEND + 4,             // [2]  MMA -> softmax
+  B_SFREE = B_SFULL + 2,            // [2]  softmax -> MMA (8 warps)
+  B_PFREE = B_SFREE + 2,            // [2]  O-CTA MMA -> S-CTA (multicast commit): P buffer consumed
+  B_PSFULL = B_PFREE + 2,           // 1    staging written (8 warps)
+  B_PSFREE = B_PSFULL + 1,          // 1    staging read by the bulk copy (1)
   // O-CTA
-  B_VFULL = B_QEND + 4,             // [4]
-  B_VEMPTY = B_VFULL + kVSlots,     // [4]
-  B_PFULL = B_VEMPTY + kVSlots,     // [2]  S-CTA softmax -> O-CTA (128 remote arrivals)
-  B_OREADY = B_PFULL + 2,           // [2]  correction warps -> MMA (4 warps)
+  B_VFULL = B_PSFREE + 1,           // [4]  cp.async arrivals of one producer group
+  B_VEMPTY = B_VFULL + kVSlots,     // [4]  MMA commit
+  B_PFULL = B_VEMPTY + kVSlots,     // [2]  one remote arrival + the P block's bytes
+  B_OREADY = B_PFULL + 2,           // [2]  correction warps -> MMA (8 warps)
   B_ODONE = B_OREADY + 2,           // 1    MMA -> correction warps (once per tile)
   B_OFINAL = B_ODONE + 1,           // 1    MMA -> epilogue (once, after the last tile)
   B_STATS = B_OFINAL + 1,           // 1    S-CTA softmax -> O-CTA epilogue (128 remote arrivals)
@@ -174,20 +187,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       mbar_init(&bar[B_QROPE], 1);
       mbar_init(&bar[B_QCONS], kSoftWarps);
-      for (int i = 0; i < 8; ++i) mbar_init(&bar[B_QRED + i], 4);
-      for (int i = 0; i < 4; ++i) mbar_init(&bar[B_QEND + i], 4);
+      for (int i = 0; i < 8; ++i) mbar_init(&bar[B_QRED + i], kSubs);
+      for (int i = 0; i < 4; ++i) mbar_init(&bar[B_QEND + i], kSubs);
       for (int i = 0; i < 2; ++i) {
         mbar_init(&bar[B_SFULL + i], 1);
         mbar_init(&bar[B_SFREE + i], kSoftWarps);
         mbar_init(&bar[B_PFREE + i], 1);
       }
+      mbar_init(&bar[B_PSFULL], kSoftWarps);
+      mbar_init(&bar[B_PSFREE], 1);
     } else {
       for (int i = 0; i < kVSlots; ++i) {
         mbar_init(&bar[B_VFULL + i], 32 * kOGroupWarps);
         mbar_init(&bar[B_VEMPTY + i], 1);
       }
       for (int i = 0; i < 2; ++i) {
-        mbar_init(&bar[B_PFULL + i], kSoftWarps);
+        mbar_init(&bar[B_PFULL + i], 1);
         mbar_init(&bar[B_OREADY + i], kSoftWarps);
       }
       mbar_init(&bar[B_ODONE], 1);
@@ -228,7 +243,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int quad = warp & 3;
-  const int sub = (warp - kSoftWarp0) >> 2;  // softmax / correction warps: which quarter of the columns
+  const int sub = (warp - kSoftWarp0) >> 2;  // softmax / correction warps: which column half
   const int h = quad * 32 + lane;
   const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
 
@@ -242,8 +257,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0 && ntiles > 0) {  // Q: 9 boxes of 128 heads x 64 dims (rope -> its own slot)
       tma_prefetch_desc(&qmap);
       mbar_arrive_expect_tx(&bar[B_QROPE], 9 * kBlk);
-      for (int blk = 0; blk < 8; ++blk)
-        tma_load_2d(base + Smem::kKRing + blk * kBlk, &qmap, 64 * blk, t * H, &bar[B_QROPE]);
+      for (int blk = 0; blk < 8; ++blk)  // dims 0..511 go through the ring and the PStage area
+        tma_load_2d(base + (blk < kKSlots ? Smem::kKRing + blk * kBlk : Smem::kPStage + (blk - kKSlots) * kBlk),
+                    &qmap, 64 * blk, t * H, &bar[B_QROPE]);
       tma_load_2d(base + Smem::kQRope, &qmap, 512, t * H, &bar[B_QROPE]);
     }
   }
@@ -254,11 +270,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (is_s) {
     if (warp < kProdWarps) {
-      // ---------- S-CTA producers: group g fills units g, g+4, ... (128 keys x 64 dims each) ----------
-      // lane l of warp w of the group copies 16-byte chunk (l & 7) of rows 4j + (l >> 3) + 32 w'
+      // ---------- S-CTA producers: group g fills units g, g+5, ... (128 keys x 64 dims each) ----------
+      // lane l of warp wg copies 16-byte chunk (l & 7) of rows 4j + (l >> 3) of its quarter of the unit
       const int g = warp / kSGroupWarps, wg = warp % kSGroupWarps;
       bool ok = ntiles == 0 || mbar_wait(&bar[B_QCONS], 0, p.status, kDevErrTimeout);
-      const kv_t* kv = p.kv;
       for (int u = g; u < ntiles * 9 && ok; u += kSGroups) {
         const int i = u / 9, blk = u % 9, slot = u % kKSlots;
         ok = mbar_wait(&bar[B_KEMPTY + slot], ((u / kKSlots) & 1) ^ 1, p.status, kDevErrTimeout);
@@ -269,7 +284,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int j = 0; j < kTile / (4 * kSGroupWarps); ++j) {
           const int r = (wg * (kTile / kSGroupWarps)) + 4 * j + (lane >> 3);
           const int prow = max(rows[i * kTile + r], 0);
-          cp_async_16(sbase + r * 128 + ((c ^ (r & 7)) << 4), kv + static_cast<int64_t>(prow) * kRowBytes + blk * 128 + c * 16);
+          cp_async_16(sbase + r * 128 + ((c ^ (r & 7)) << 4), p.kv + static_cast<int64_t>(prow) * kRowBytes + blk * 128 + c * 16);
         }
         cp_async_mbar_arrive_noinc(&bar[B_KFULL + slot]);
       }
@@ -311,24 +326,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
       __syncwarp();
+    } else if (warp == kCopyWarp) {
+      // ---------- S-CTA copier: staging -> the O-CTA's P buffer i & 1, one bulk copy per tile ----------
+      if (lane == 0 && ntiles > 0) {
+        const uint8_t* stage = base + Smem::kPStage;
+        const uint32_t peer_p = peer_addr(smem_u32(base + Smem::kP), 1);
+        const uint32_t peer_pfull = peer_addr(smem_u32(&bar[B_PFULL]), 1);
+        bool ok = true;
+        for (int i = 0; i < ntiles && ok; ++i) {
+          const int sb = i & 1;
+          // all eight softmax warps wrote block i, and the O-CTA's MMA of tile i - 2 released buffer sb
+          ok = mbar_wait(&bar[B_PSFULL], i & 1, p.status, kDevErrTimeout) &&
+               mbar_wait(&bar[B_PFREE + sb], ((i >> 1) & 1) ^ 1, p.status, kDevErrTimeout);
+          if (!ok) break;
+          mbar_arrive_expect_tx_remote(peer_pfull + static_cast<uint32_t>(sb * 8), kPShip);
+          bulk_copy_to_peer(peer_p + static_cast<uint32_t>(sb * kPStride), stage, kPShip,
+                            peer_pfull + static_cast<uint32_t>(sb * 8));
+          bulk_commit_group();
+          bulk_wait_read_all();  // the staging buffer may be rewritten
+          mbar_arrive(&bar[B_PSFREE]);
+        }
+        // the O-CTA's last multicast commits land in this CTA's barriers: wait for them before exit
+        if (ok) {
+          const int i1 = ntiles - 1;
+          mbar_wait(&bar[B_PFREE + (i1 & 1)], (i1 >> 1) & 1, p.status, kDevErrTimeout);
+          if (ntiles > 1) mbar_wait(&bar[B_PFREE + ((i1 - 1) & 1)], ((i1 - 1) >> 1) & 1, p.status, kDevErrTimeout);
+        }
+      }
+      __syncwarp();
     } else {
-      // ---------- S-CTA softmax (warps 15..30: thread = head h, keys 32*sub .. 32*sub+31) ----------
-      const uint32_t peer_p = peer_addr(smem_u32(base + Smem::kP), 1);
-      const uint32_t peer_alpha = peer_addr(smem_u32(base + Smem::kAlpha), 1);
-      const uint32_t peer_flags = peer_addr(smem_u32(base + Smem::kFlags), 1);
-      const uint32_t peer_stats = peer_addr(smem_u32(base + Smem::kStats), 1);
-      const uint32_t peer_pfull = peer_addr(smem_u32(&bar[B_PFULL]), 1);
-      const uint32_t peer_statbar = peer_addr(smem_u32(&bar[B_STATS]), 1);
-      float* red = reinterpret_cast<float*>(base + Smem::kRed);    // [2][4][128]
-      float* redl = reinterpret_cast<float*>(base + Smem::kRedL);  // [2][4][128]: l, lr
+      // ---------- S-CTA softmax (warps 21..28: thread = head h, keys 64*sub .. 64*sub+63) ----------
+      float* red = reinterpret_cast<float*>(base + Smem::kRed);    // [2][kSubs][128]
+      float* redl = reinterpret_cast<float*>(base + Smem::kRedL);  // [2][kSubs][128]: l, lr
+      uint8_t* stage = base + Smem::kPStage;
       float m_ref = -INFINITY, l = 0.f, lr = 0.f;
       bool ok = true;
       if (ntiles > 0) {
-        // Q dims 0..511: swizzled blocks 2*sub, 2*sub+1 of ring slots 0..7 -> TMEM (lane = head)
+        // Q dims 0..511: blocks 4*sub .. 4*sub+3 (ring slots / PStage) -> TMEM columns (lane = head)
         ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_QROPE], 0, p.status, kDevErrTimeout));
         if (ok) {
-          for (int blk = 2 * sub; blk < 2 * sub + 2; ++blk) {
-            const uint8_t* rowp = base + Smem::kKRing + blk * kBlk + h * 128;
+          for (int blk = 4 * sub; blk < 4 * sub + 4; ++blk) {
+            const uint8_t* rowp =
+                base + (blk < kKSlots ? Smem::kKRing + blk * kBlk : Smem::kPStage + (blk - kKSlots) * kBlk) + h * 128;
             uint32_t r[32];
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -344,31 +383,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[B_QCONS]);  // ring slots 0..7 may be refilled
+        if (lane == 0) mbar_arrive(&bar[B_QCONS]);  // ring slots may be refilled
       }
       for (int i = 0; i < ntiles && ok; ++i) {
         const int sb = i & 1;
         ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_SFULL + sb], (i >> 1) & 1, p.status, kDevErrTimeout));
         if (!ok) break;
         tc_fence_after();
-        uint32_t v[32];
-        tmem_ld32_sync(tmem + lane_base + kColS + kTile * sb + 32 * sub, v);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[B_SFREE + sb]);
-        const uint32_t m = masks[4 * i + sub];
+        const uint32_t srow = tmem + lane_base + kColS + kTile * sb + 64 * sub;
+        // pass 1: maximum over this warp's 64 keys (scaled, log2 units)
         float pmax = -INFINITY;
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          uint32_t v[32];
+          tmem_ld32_sync(srow + 32 * c, v);
+          const uint32_t m = masks[4 * i + 2 * sub + c];
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if ((m >> j) & 1u) pmax = fmaxf(pmax, __uint_as_float(v[j]) * p.scale_log2);
-        // tile maximum of head h across the four warps of this quadrant (shared memory + mbarrier)
-        red[(sb * 4 + sub) * 128 + h] = pmax;
+          for (int j = 0; j < 32; ++j)
+            if ((m >> j) & 1u) pmax = fmaxf(pmax, __uint_as_float(v[j]) * p.scale_log2);
+        }
+        // tile maximum of head h across this quadrant's warps (shared memory + mbarrier)
+        red[(sb * kSubs + sub) * 128 + h] = pmax;
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[B_QRED + sb * 4 + quad]);
         ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_QRED + sb * 4 + quad], (i >> 1) & 1, p.status, kDevErrTimeout));
         if (!ok) break;
-        const float tmax = fmaxf(fmaxf(red[(sb * 4 + 0) * 128 + h], red[(sb * 4 + 1) * 128 + h]),
-                                 fmaxf(red[(sb * 4 + 2) * 128 + h], red[(sb * 4 + 3) * 128 + h]));
+        float tmax = -INFINITY;
+#pragma unroll
+        for (int s2 = 0; s2 < kSubs; ++s2) tmax = fmaxf(tmax, red[(sb * kSubs + s2) * 128 + h]);
         const bool need = tmax > m_ref + kRescaleThreshold;
         const float alpha = need ? exp2f(m_ref - tmax) : 1.f;  // 0 when m_ref is -inf
         if (need) {
@@ -376,72 +418,75 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           lr *= alpha;
           m_ref = tmax;
         }
-        const bool warp_rescale = __any_sync(0xffffffffu, need && i > 0);
-        // the O-CTA must be done with the P buffer of tile i-2
-        ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_PFREE + sb], ((i >> 1) & 1) ^ 1, p.status, kDevErrTimeout));
+        const bool quad_rescale = __any_sync(0xffffffffu, need && i > 0);
+        // the previous P block must have left the staging buffer
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_PSFREE], (i & 1) ^ 1, p.status, kDevErrTimeout));
         if (!ok) break;
-        // P[h, 32*sub .. +31] (bf16) into the peer's K-major swizzled buffer (2 blocks of 64 keys)
+        // pass 2: P[h, 64*sub .. +63] (bf16) into the staging copy of the peer's K-major swizzled
+        // P buffer: block sub (64 keys), chunks of 8 keys XOR-swizzled by head
         const float m_use = (m_ref > -INFINITY) ? m_ref : 0.f;  // m_ref = -inf: every key so far masked
-        const uint32_t prow = peer_p + static_cast<uint32_t>(sb * 2 * kBlk + h * 128);
+        uint8_t* prow = stage + sub * kBlk + h * 128;
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          uint32_t v[32];
+          tmem_ld32_sync(srow + 32 * c, v);
+          const uint32_t m = masks[4 * i + 2 * sub + c];
 #pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {  // 8 keys = one 16-byte chunk
-          uint32_t w[4];
+          for (int q8 = 0; q8 < 4; ++q8) {  // 8 keys = one 16-byte chunk
+            uint32_t w[4];
 #pragma unroll
-          for (int q2 = 0; q2 < 4; ++q2) {
-            const int j0 = 8 * q8 + 2 * q2;
-            const float p0 = ((m >> j0) & 1u) ? fast_exp2(fmaf(__uint_as_float(v[j0]), p.scale_log2, -m_use)) : 0.f;
-            const float p1 = ((m >> (j0 + 1)) & 1u) ? fast_exp2(fmaf(__uint_as_float(v[j0 + 1]), p.scale_log2, -m_use)) : 0.f;
-            const __nv_bfloat162 bp = __floats2bfloat162_rn(p0, p1);
-            l += p0 + p1;
-            lr += __low2float(bp) + __high2float(bp);
-            w[q2] = *reinterpret_cast<const uint32_t*>(&bp);
+            for (int q2 = 0; q2 < 4; ++q2) {
+              const int j0 = 8 * q8 + 2 * q2;
+              const float p0 = ((m >> j0) & 1u) ? fast_exp2(fmaf(__uint_as_float(v[j0]), p.scale_log2, -m_use)) : 0.f;
+              const float p1 = ((m >> (j0 + 1)) & 1u) ? fast_exp2(fmaf(__uint_as_float(v[j0 + 1]), p.scale_log2, -m_use)) : 0.f;
+              const __nv_bfloat162 bp = __floats2bfloat162_rn(p0, p1);
+              l += p0 + p1;
+              lr += __low2float(bp) + __high2float(bp);
+              w[q2] = *reinterpret_cast<const uint32_t*>(&bp);
+            }
+            const int chunk = 4 * c + q8;  // chunk 0..7 within block `sub`
+            *reinterpret_cast<uint4*>(prow + (((chunk ^ (h & 7))) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
           }
-          const int chunk = 4 * sub + q8;  // 0..15: block chunk>>3, chunk-in-block chunk&7
-          st_cluster_v4(prow + static_cast<uint32_t>((chunk >> 3) * kBlk + (((chunk & 7) ^ (h & 7)) << 4)), w[0], w[1],
-                        w[2], w[3]);
         }
-        if (sub == 0) {
-          st_cluster_f32(peer_alpha + static_cast<uint32_t>((sb * 128 + h) * 4), alpha);
-          if (lane == 0) st_cluster_u32(peer_flags + static_cast<uint32_t>((sb * 4 + quad) * 4), warp_rescale ? 1u : 0u);
-        }
-        fence_proxy_async_cluster();
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(peer_pfull + static_cast<uint32_t>(sb * 8));
+        if (lane == 0) mbar_arrive(&bar[B_SFREE + sb]);
+        if (sub == 0) {
+          reinterpret_cast<float*>(stage + kPAlpha)[h] = alpha;
+          if (lane == 0) reinterpret_cast<uint32_t*>(stage + kPFlags)[quad] = quad_rescale ? 1u : 0u;
+        }
+        fence_proxy_async_smem();  // staging writes (generic proxy) -> bulk copy reads (async proxy)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[B_PSFULL]);
       }
-      // per-head sums over the four warps of the quadrant, then the final statistics (always sent,
-      // so the O-CTA never waits in vain)
-      redl[(0 * 4 + sub) * 128 + h] = l;
-      redl[(1 * 4 + sub) * 128 + h] = lr;
+      // per-head sums over the quadrant's warps, then the final statistics (always sent, so the
+      // O-CTA never waits in vain)
+      redl[(0 * kSubs + sub) * 128 + h] = l;
+      redl[(1 * kSubs + sub) * 128 + h] = lr;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[B_QEND + quad]);
       const bool sums_ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_QEND + quad], 0, p.status, kDevErrTimeout));
       if (sub == 0) {
         float lt = 0.f, lrt = 0.f;
         if (sums_ok) {
-          for (int q = 0; q < 4; ++q) {
-            lt += redl[(0 * 4 + q) * 128 + h];
-            lrt += redl[(1 * 4 + q) * 128 + h];
+          for (int s2 = 0; s2 < kSubs; ++s2) {
+            lt += redl[(0 * kSubs + s2) * 128 + h];
+            lrt += redl[(1 * kSubs + s2) * 128 + h];
           }
         }
+        const uint32_t peer_stats = peer_addr(smem_u32(base + Smem::kStats), 1);
         st_cluster_f32(peer_stats + static_cast<uint32_t>(h * 4), m_ref);
         st_cluster_f32(peer_stats + static_cast<uint32_t>((128 + h) * 4), lt);
         st_cluster_f32(peer_stats + static_cast<uint32_t>((256 + h) * 4), lrt);
-        mbar_arrive_remote(peer_statbar);
-      }
-      // the last multicast commits of the O-CTA land in this CTA's barriers: wait for them
-      if (ok && ntiles > 0) {
-        const int i1 = ntiles - 1;
-        mbar_wait(&bar[B_PFREE + (i1 & 1)], (i1 >> 1) & 1, p.status, kDevErrTimeout);
-        if (ntiles > 1) mbar_wait(&bar[B_PFREE + ((i1 - 1) & 1)], ((i1 - 1) >> 1) & 1, p.status, kDevErrTimeout);
+        mbar_arrive_remote(peer_addr(smem_u32(&bar[B_STATS]), 1));
       }
     }
   } else {
     if (warp < kProdWarps) {
       // ---------- O-CTA producers: V in units of 128 keys x 128 dims (2 blocks), one unit per group ----
-      // lane l copies 16-byte chunk (l & 15) of rows 2j + (l >> 4) of its warp's quarter of the unit
+      // lane l copies 16-byte chunk (l & 15) of rows r_lo + 2j + (l >> 4) of its warp's share of the unit
       const int g = warp / kOGroupWarps, wg = warp % kOGroupWarps;
       const int r_lo = (wg * kTile) / kOGroupWarps, r_hi = ((wg + 1) * kTile) / kOGroupWarps;
-      const kv_t* kv = p.kv;
       bool ok = true;
       for (int u = g; u < ntiles * 4 && ok; u += kOGroups) {
         const int i = u / 4, qd = u % 4, slot = u % kVSlots;
@@ -453,7 +498,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int r = r_lo + (lane >> 4); r < r_hi; r += 2) {  // 16 lanes per 256-byte row segment
           const int prow = max(rows[i * kTile + r], 0);
           cp_async_16(sbase + (c >> 3) * kBlk + r * 128 + (((c & 7) ^ (r & 7)) << 4),
-                      kv + static_cast<int64_t>(prow) * kRowBytes + qd * 256 + c * 16);
+                      p.kv + static_cast<int64_t>(prow) * kRowBytes + qd * 256 + c * 16);
         }
         cp_async_mbar_arrive_noinc(&bar[B_VFULL + slot]);
       }
@@ -471,7 +516,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                mbar_wait_cluster(&bar[B_PFULL + pb], (i >> 1) & 1, p.status, kDevErrTimeout);
           if (!ok) break;
           tc_fence_after();
-          const uint64_t pd = pdesc0 + static_cast<uint64_t>((pb * 2 * kBlk) >> 4);
+          const uint64_t pd = pdesc0 + static_cast<uint64_t>((pb * kPStride) >> 4);
           for (int qd = 0; qd < 4; ++qd) {
             const int u = i * 4 + qd, slot = u % kVSlots;
             ok = mbar_wait(&bar[B_VFULL + slot], (u / kVSlots) & 1, p.status, kDevErrTimeout);
@@ -494,26 +539,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
       __syncwarp();
-    } else {
-      // ---------- O-CTA correction + epilogue (warps 15..30: head h, O columns 128*sub .. +127) -------
-      const float* alpha_s = reinterpret_cast<const float*>(base + Smem::kAlpha);
-      const volatile uint32_t* flags = reinterpret_cast<const volatile uint32_t*>(base + Smem::kFlags);
+    } else if (warp < kCopyWarp) {
+      // ---------- O-CTA correction + epilogue (warps 21..28: head h, O columns 256*sub .. +255) ------
       const volatile float* stats = reinterpret_cast<const volatile float*>(base + Smem::kStats);
-      const uint32_t ocol = tmem + lane_base + kColO + 128 * sub;
+      const uint32_t ocol = tmem + lane_base + kColO + 256 * sub;
       bool ok = true;
       for (int i = 0; i < ntiles && ok; ++i) {
         const int pb = i & 1;
         ok = __all_sync(0xffffffffu, mbar_wait_cluster(&bar[B_PFULL + pb], (i >> 1) & 1, p.status, kDevErrTimeout));
         if (!ok) break;
-        if (flags[pb * 4 + quad] != 0u) {
-          // P(i) was written after MMA2(i-2) completed, so B_ODONE is at most one phase behind:
+        const uint8_t* pblk = base + Smem::kP + pb * kPStride;
+        if (reinterpret_cast<const volatile uint32_t*>(pblk + kPFlags)[quad] != 0u) {
+          // P(i) was shipped after MMA2(i-2) completed, so B_ODONE is at most one phase behind:
           // the parity wait below really waits for MMA2(i-1).
           ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_ODONE], (i - 1) & 1, p.status, kDevErrTimeout));
           if (!ok) break;
           tc_fence_after();
-          const float a = alpha_s[pb * 128 + h];
+          const float a = reinterpret_cast<const float*>(pblk + kPAlpha)[h];
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < 8; ++c) {
             uint32_t o[32];
             tmem_ld32_sync(ocol + 32 * c, o);
 #pragma unroll
@@ -537,9 +581,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const float inv = (have_o && lr > 0.f) ? 1.f / lr : 0.f;
       const float lse_nat = (have_o && l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
       if (p.nsplit == 1) {
-        uint16_t* dst = p.out + (static_cast<int64_t>(t) * H + h) * kDV + 128 * sub;
+        uint16_t* dst = p.out + (static_cast<int64_t>(t) * H + h) * kDV + 256 * sub;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 8; ++c) {
           uint32_t o[32];
           if (have_o) {
             tmem_ld32_sync(ocol + 32 * c, o);
@@ -563,9 +607,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (sub == 0 && h < H && p.lse) p.lse[static_cast<int64_t>(t) * H + h] = lse_nat;
       } else {
         const int64_t prow = (static_cast<int64_t>(t) * p.nsplit + split) * H + h;
-        float* dst = p.part_o + prow * kDV + 128 * sub;
+        float* dst = p.part_o + prow * kDV + 256 * sub;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 8; ++c) {
           uint32_t o[32];
           if (have_o) {
             tmem_ld32_sync(ocol + 32 * c, o);
