@@ -100,7 +100,8 @@ dsa_status_t dsa_index_scores(const dsa_batch_t* batch, const void* plan, const 
                               const float* kI_scale, float* scores, int64_t ld, void* stream);
 
 /* ---- step 2: top-k ----------------------------------------------------------------------
- * scores f32 [T, ld] as written by dsa_index_scores (row t read at j <= p only).
+ * scores f32 [T, ld] as written by dsa_index_scores (row t read at j <= p only); ld % 4 == 0,
+ *        ld >= max_seq_len. max_seq_len <= 262144 (else DSA_ERR_UNSUPPORTED).
  * S      int32 [T, k] out: the min(k, p+1) positions with the largest scores, followed by -1.
  *        Among equal scores the smaller position wins. Selected positions are listed in
  *        increasing position order. 1 <= k <= 4096. */

@@ -119,8 +119,9 @@ dsa_status_t dsa_topk(const dsa_batch_t* batch, const void* plan, const float* s
   if (st != DSA_OK) return st;
   if (k < 1 || k > kMaxTopK) return DSA_ERR_UNSUPPORTED;
   if (batch->total_q == 0) return DSA_OK;
-  if (!plan || !scores || !S || !aligned16(plan)) return DSA_ERR_INVALID_ARG;
-  if (ld < batch->max_seq_len) return DSA_ERR_INVALID_ARG;
+  if (batch->max_seq_len > kMaxTopKRow) return DSA_ERR_UNSUPPORTED;
+  if (!plan || !scores || !S || !aligned16(plan) || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
+  if (ld < batch->max_seq_len || ld % 4 != 0) return DSA_ERR_INVALID_ARG;
   return from_cuda(launch_topk(to_dev(batch), plan, scores, ld, k, S, stream));
 }
 

@@ -20,6 +20,7 @@ constexpr int kDV = DSA_D_V;             // value width
 constexpr int kIdxTileKeys = 128;        // keys per indexer MMA tile (2 pages)
 constexpr int kIdxCols = 256;            // query-head columns per indexer group (MMA N <= 256)
 constexpr int kMaxTopK = 4096;
+constexpr int kMaxTopKRow = 262144;  // longest score row the top-k kernel takes
 
 // Device status bits recorded by kernels (dsa_status_read maps them to dsa_status_t).
 constexpr uint32_t kDevErrTimeout = 1u;

@@ -12,17 +12,19 @@
 //   S-CTA (rank 0): S = Q C^T and the softmax.
 //     * Q (128 heads x 576 bf16): dims 0..511 in TMEM as the A operand (256 columns), the 64 rope
 //       dims in shared memory (one 128-byte-swizzled block).
-//     * 20 producer warps gather the selected latent rows with 16-byte cp.async (8 lanes per
-//       128-byte row segment, XOR-swizzled on the way into the canonical 128-byte-swizzled K-major
-//       UMMA layout) into a 10-slot ring of 128 keys x 64 dims. Random 1152-byte rows need
-//       hundreds of loads in flight per SM; TMA gather4 tops out near 2 TB/s (per-copy cost).
+//     * 20 producer warps gather latent dims 0..511 of the selected rows with 16-byte cp.async (8
+//       lanes per 128-byte row segment, XOR-swizzled on the way into the canonical 128-byte-swizzled
+//       K-major UMMA layout) into an 8-slot ring (slot = 64-dim block of the current tile); a ninth
+//       warp fetches the rope dims 512..575 with TMA gather4 (4 rows per copy) into a 2-slot ring.
+//       Random 1152-byte rows need hundreds of loads in flight per SM; the TMA engine runs beside
+//       the load/store unit and adds to the rate one SM reaches with cp.async alone.
 //     * Each tile of 128 keys costs 36 tcgen05.mma (M=128 heads, N=128 keys, K=16), which run at
 //       the full bf16 rate; S tiles are double-buffered in TMEM (2 x 128 columns).
 //     * Eight softmax warps (two per TMEM lane quadrant, 64 keys each) read S twice (maximum, then
 //       exponentials), keep an online softmax whose reference maximum only moves when a tile's
 //       maximum exceeds it by more than 2^8, and write bf16 P, the per-head rescale factors and
-//       per-quadrant rescale flags into a local staging buffer; a copier warp ships the 33 KB block
-//       to the O-CTA with a single bulk copy that completes on the O-CTA's barrier.
+//       per-quadrant rescale flags straight into the O-CTA's shared memory with st.async, whose
+//       bytes complete the O-CTA's barrier for that P buffer (two buffers, alternating by tile).
 //   O-CTA (rank 1): O = P V.
 //     * O (128 heads x 512 fp32) fills its whole TMEM. V = c[0:512] of the same rows (mostly L2
 //       hits: the S-CTA fetched them) is gathered by 20 producer warps in units of 128 keys x 128
@@ -30,7 +32,7 @@
 //     * Per tile: 32 tcgen05.mma (M=128, N=128 dims, K=16 keys), A = P (shared memory, K-major),
 //       B = V (MN-major). Completion is multicast back to the S-CTA to free the P buffer.
 //     * Eight correction warps rescale O rows in TMEM when a quadrant is flagged (rare), and at
-//       the end normalise O and write the output.
+//       the end normalise O; the bf16 rows are staged in shared memory and leave with TMA stores.
 //
 // Splits (several clusters over one S_t) write normalised partial outputs and their log-sum-exp
 // to the workspace; a combine kernel merges them: o = sum_s exp(lse_s - lse) o_s.
@@ -38,6 +40,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstring>
 
 #include "dsa_internal.h"
 #include "dsa_ptx.cuh"
@@ -46,6 +49,8 @@ namespace dsa {
 
 int make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* ptr, uint64_t inner,
                  uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows);
+int make_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2,
+                 uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1, uint32_t b2);
 
 namespace {
 
@@ -54,20 +59,22 @@ constexpr int kTile = 128;                   // keys per tile (MMA N for S, K-ex
 constexpr int kMaxKeysPerCta = 2048;         // S_t entries one cluster handles
 constexpr int kMaxTiles = kMaxKeysPerCta / kTile;
 constexpr int kBlk = kTile * 128;            // 128 keys x 64 dims bf16 = 16 KB
-constexpr int kKSlots = 10;                  // S-CTA ring slots (one 64-dim block of one tile each)
+constexpr int kKSlots = 8;                   // S-CTA cp.async ring: latent blocks 0..7 of a tile, slot = block
+constexpr int kRSlots = 2;                   // S-CTA TMA ring: the rope block (dims 512..575) of a tile
 constexpr int kVSlots = 4;                   // O-CTA ring slots (two 64-dim blocks of one tile each)
-constexpr int kProdWarps = 20;               // warps 0..19: gather producers
+constexpr int kProdWarps = 20;               // warps 0..19: cp.async gather producers
 // A producer group fills one ring unit at a time; each ring slot belongs to exactly one group
 // (slot % groups == group), so a group never runs two uses ahead of the consumer on a slot's
 // barrier, which a parity wait could not tell from one use ahead.
-constexpr int kSGroupWarps = 4, kSGroups = kProdWarps / kSGroupWarps;  // S-CTA: 5 groups, 10 slots
+constexpr int kSGroupWarps = 5, kSGroups = kProdWarps / kSGroupWarps;  // S-CTA: 4 groups, 8 slots
 constexpr int kOGroupWarps = 5, kOGroups = kProdWarps / kOGroupWarps;  // O-CTA: 4 groups, 4 slots
 constexpr int kMmaWarp = kProdWarps;         // warp 20: TMEM allocator and MMA issuer
 constexpr int kSoftWarp0 = kProdWarps + 1;   // warps 21..28: softmax (S-CTA) / correction (O-CTA),
 constexpr int kSoftWarps = 8;                //   two per TMEM lane quadrant
 constexpr int kSubs = kSoftWarps / 4;        // column halves per quadrant
-constexpr int kCopyWarp = kSoftWarp0 + kSoftWarps;  // warp 29: ships P blocks (S-CTA only)
-constexpr int kThreads = 32 * (kCopyWarp + 1);
+constexpr int kRopeWarp = kSoftWarp0 + kSoftWarps;  // warp 29: rope blocks by TMA gather4 (S-CTA only)
+constexpr int kThreads = 32 * (kRopeWarp + 1);
+constexpr int kRowIters = (kMaxKeysPerCta + kThreads - 1) / kThreads;
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
 
 // TMEM columns
@@ -86,14 +93,14 @@ constexpr int kPStride = 33 * 1024;          // keeps every P block 1024-byte al
 struct Smem {
   // S-CTA
   static constexpr int kQRope = 0;                               // 16 KB
-  static constexpr int kKRing = kQRope + kBlk;                   // 10 x 16 KB
-  static constexpr int kPStage = kKRing + kKSlots * kBlk;        // one P block being assembled
-  static constexpr int kRed = kPStage + kPStride;                // float [2][kSubs][128]: tile maxima
+  static constexpr int kKRing = kQRope + kBlk;                   // 8 x 16 KB (Q dims 0..511 at start)
+  static constexpr int kRRing = kKRing + kKSlots * kBlk;         // 2 x 16 KB
+  static constexpr int kRed = kRRing + kRSlots * kBlk;           // float [2][kSubs][128]: tile maxima
   static constexpr int kRedL = kRed + 2 * kSubs * 128 * 4;       // float [2][kSubs][128]: l, lr
   static constexpr int kSEnd = kRedL + 2 * kSubs * 128 * 4;
   // O-CTA
   static constexpr int kP = 0;                                   // 2 P blocks, kPStride apart
-  static constexpr int kVRing = kP + 2 * kPStride;               // 4 x 32 KB
+  static constexpr int kVRing = kP + 2 * kPStride;               // 4 x 32 KB; output staging at the end
   static constexpr int kStats = kVRing + kVSlots * 2 * kBlk;     // float [3][128]: m, l, lr
   static constexpr int kOEnd = kStats + 3 * 128 * 4;
   // both
@@ -109,27 +116,27 @@ struct Smem {
 static_assert(Smem::kDynamic <= 232448, "sparse MLA shared memory exceeds the 227 KB limit");
 static_assert(kPShip <= kPStride && kPShip % 16 == 0, "P block");
 static_assert(kKSlots % kSGroups == 0 && kVSlots % kOGroups == 0, "every ring slot needs a single owner group");
-static_assert(kTile % (4 * kSGroupWarps) == 0, "S-CTA rows per warp");
+static_assert(kKSlots == 8, "one cp.async slot per latent block of a tile");
 static_assert(kTile == 32 * 2 * kSubs, "softmax warps cover a tile");
 
 // barrier indices (same offsets in both CTAs; each CTA initialises the ones it owns)
 enum : int {
   // S-CTA
-  B_KFULL = 0,                      // [10] cp.async arrivals of one producer group
-  B_KEMPTY = B_KFULL + kKSlots,     // [10] MMA commit
-  B_QROPE = B_KEMPTY + kKSlots,     // 1    TMA of Q
+  B_KFULL = 0,                      // [8]  cp.async arrivals of one producer group
+  B_KEMPTY = B_KFULL + kKSlots,     // [8]  MMA commit
+  B_RFULL = B_KEMPTY + kKSlots,     // [2]  TMA bytes of a rope block
+  B_REMPTY = B_RFULL + kRSlots,     // [2]  MMA commit
+  B_QROPE = B_REMPTY + kRSlots,     // 1    TMA of Q
   B_QCONS = B_QROPE + 1,            // 1    softmax warps moved Q out of the ring (8 warps)
   B_QRED = B_QCONS + 1,             // [2][4] partial maxima of one quadrant written (kSubs warps)
   B_QEND = B_QRED + 8,              // [4]  partial sums of one quadrant written (kSubs warps)
   B_SFULL = B_QEND + 4,             // [2]  MMA -> softmax
   B_SFREE = B_SFULL + 2,            // [2]  softmax -> MMA (8 warps)
   B_PFREE = B_SFREE + 2,            // [2]  O-CTA MMA -> S-CTA (multicast commit): P buffer consumed
-  B_PSFULL = B_PFREE + 2,           // 1    staging written (8 warps)
-  B_PSFREE = B_PSFULL + 1,          // 1    staging read by the bulk copy (1)
   // O-CTA
-  B_VFULL = B_PSFREE + 1,           // [4]  cp.async arrivals of one producer group
+  B_VFULL = B_PFREE + 2,            // [4]  cp.async arrivals of one producer group
   B_VEMPTY = B_VFULL + kVSlots,     // [4]  MMA commit
-  B_PFULL = B_VEMPTY + kVSlots,     // [2]  one remote arrival + the P block's bytes
+  B_PFULL = B_VEMPTY + kVSlots,     // [2]  one remote arrival + the P block's bytes (st.async)
   B_OREADY = B_PFULL + 2,           // [2]  correction warps -> MMA (8 warps)
   B_ODONE = B_OREADY + 2,           // 1    MMA -> correction warps (once per tile)
   B_OFINAL = B_ODONE + 1,           // 1    MMA -> epilogue (once, after the last tile)
@@ -158,7 +165,8 @@ struct MlaParams {
 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    sparse_mla_kernel(const __grid_constant__ CUtensorMap qmap, const MlaParams p) {
+    sparse_mla_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kvmap,
+                      const __grid_constant__ CUtensorMap omap, const MlaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   int32_t* rows = reinterpret_cast<int32_t*>(base + Smem::kRows);
@@ -185,6 +193,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mbar_init(&bar[B_KFULL + i], 32 * kSGroupWarps);  // one cp.async arrival per producer lane
         mbar_init(&bar[B_KEMPTY + i], 1);
       }
+      for (int i = 0; i < kRSlots; ++i) {
+        mbar_init(&bar[B_RFULL + i], 1);
+        mbar_init(&bar[B_REMPTY + i], 1);
+      }
       mbar_init(&bar[B_QROPE], 1);
       mbar_init(&bar[B_QCONS], kSoftWarps);
       for (int i = 0; i < 8; ++i) mbar_init(&bar[B_QRED + i], kSubs);
@@ -194,8 +206,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mbar_init(&bar[B_SFREE + i], kSoftWarps);
         mbar_init(&bar[B_PFREE + i], 1);
       }
-      mbar_init(&bar[B_PSFULL], kSoftWarps);
-      mbar_init(&bar[B_PSFREE], 1);
     } else {
       for (int i = 0; i < kVSlots; ++i) {
         mbar_init(&bar[B_VFULL + i], 32 * kOGroupWarps);
@@ -210,6 +220,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&bar[B_STATS], 128);
     }
     fence_barrier_init();
+    if (is_s && ntiles > 0) {  // Q: 9 boxes of 128 heads x 64 dims; dims 0..511 land in the cp.async ring
+      tma_prefetch_desc(&qmap);
+      mbar_arrive_expect_tx(&bar[B_QROPE], 9 * kBlk);
+      for (int blk = 0; blk < 8; ++blk) tma_load_2d(base + Smem::kKRing + blk * kBlk, &qmap, 64 * blk, t * H, &bar[B_QROPE]);
+      tma_load_2d(base + Smem::kQRope, &qmap, 512, t * H, &bar[B_QROPE]);
+    }
   }
   if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, 512);
@@ -220,23 +236,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int32_t* S_row = p.S + static_cast<int64_t>(t) * p.k + e0;
   const int32_t* bt_row = p.bd.block_table + static_cast<int64_t>(b) * p.bd.max_pages;
   const int n_b = __ldg(p.bd.seq_lens + b);
-  for (int e = threadIdx.x; e < ntiles * kTile; e += kThreads) {
-    int r = -1;
-    if (e < nkeys) {
-      const int j = __ldg(S_row + e);
-      if (j >= 0) {
-        if (j > pos || j >= n_b) {
-          report_error(p.status, kDevErrIndex);
-        } else {
-          const int pg = __ldg(bt_row + j / kPage);
-          if (pg < 0 || pg >= p.bd.num_pages)
+  {
+    // all index loads first, then all page lookups: two dependent round trips to memory in total
+    int jv[kRowIters], pg[kRowIters];
+#pragma unroll
+    for (int it = 0; it < kRowIters; ++it) {
+      const int e = threadIdx.x + it * kThreads;
+      jv[it] = (e < nkeys) ? __ldg(S_row + e) : -1;
+    }
+#pragma unroll
+    for (int it = 0; it < kRowIters; ++it) {
+      const int j = jv[it];
+      const bool in_range = j >= 0 && j <= pos && j < n_b;
+      if (j >= 0 && !in_range) report_error(p.status, kDevErrIndex);
+      pg[it] = in_range ? __ldg(bt_row + j / kPage) : -1;
+      if (!in_range) jv[it] = -1;
+    }
+#pragma unroll
+    for (int it = 0; it < kRowIters; ++it) {
+      const int e = threadIdx.x + it * kThreads;
+      if (e < ntiles * kTile) {
+        int r = -1;
+        if (jv[it] >= 0) {
+          if (pg[it] < 0 || pg[it] >= p.bd.num_pages)
             report_error(p.status, kDevErrIndex);
           else
-            r = pg * kPage + (j % kPage);
+            r = pg[it] * kPage + (jv[it] % kPage);
         }
+        rows[e] = r;
       }
     }
-    rows[e] = r;
   }
   tc_fence_before();
   __syncthreads();
@@ -254,14 +283,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 32; ++c) m |= (rows[i * kTile + 32 * w + c] >= 0 ? 1u : 0u) << c;
       masks[threadIdx.x] = m;
     }
-    if (threadIdx.x == 0 && ntiles > 0) {  // Q: 9 boxes of 128 heads x 64 dims (rope -> its own slot)
-      tma_prefetch_desc(&qmap);
-      mbar_arrive_expect_tx(&bar[B_QROPE], 9 * kBlk);
-      for (int blk = 0; blk < 8; ++blk)  // dims 0..511 go through the ring and the PStage area
-        tma_load_2d(base + (blk < kKSlots ? Smem::kKRing + blk * kBlk : Smem::kPStage + (blk - kKSlots) * kBlk),
-                    &qmap, 64 * blk, t * H, &bar[B_QROPE]);
-      tma_load_2d(base + Smem::kQRope, &qmap, 512, t * H, &bar[B_QROPE]);
-    }
   }
   tc_fence_before();
   __syncthreads();
@@ -270,23 +291,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (is_s) {
     if (warp < kProdWarps) {
-      // ---------- S-CTA producers: group g fills units g, g+5, ... (128 keys x 64 dims each) ----------
-      // lane l of warp wg copies 16-byte chunk (l & 7) of rows 4j + (l >> 3) of its quarter of the unit
+      // ---------- S-CTA producers: latent blocks 0..7; group g fills blocks g and g + 4 of every tile ----------
+      // lane l of warp wg copies 16-byte chunk (l & 7) of rows r_lo + 4j + (l >> 3) of its fifth of the unit
       const int g = warp / kSGroupWarps, wg = warp % kSGroupWarps;
+      const int r_lo = (wg * kTile) / kSGroupWarps, r_hi = ((wg + 1) * kTile) / kSGroupWarps;
       bool ok = ntiles == 0 || mbar_wait(&bar[B_QCONS], 0, p.status, kDevErrTimeout);
-      for (int u = g; u < ntiles * 9 && ok; u += kSGroups) {
-        const int i = u / 9, blk = u % 9, slot = u % kKSlots;
-        ok = mbar_wait(&bar[B_KEMPTY + slot], ((u / kKSlots) & 1) ^ 1, p.status, kDevErrTimeout);
+      for (int u = g; u < ntiles * kKSlots && ok; u += kSGroups) {
+        const int i = u / kKSlots, blk = u % kKSlots;  // the slot is the block
+        ok = mbar_wait(&bar[B_KEMPTY + blk], (i & 1) ^ 1, p.status, kDevErrTimeout);
         if (!ok) break;
-        const uint32_t sbase = smem_u32(base + Smem::kKRing + slot * kBlk);
+        const uint32_t sbase = smem_u32(base + Smem::kKRing + blk * kBlk);
         const int c = lane & 7;
 #pragma unroll 4
-        for (int j = 0; j < kTile / (4 * kSGroupWarps); ++j) {
-          const int r = (wg * (kTile / kSGroupWarps)) + 4 * j + (lane >> 3);
+        for (int r = r_lo + (lane >> 3); r < r_hi; r += 4) {
           const int prow = max(rows[i * kTile + r], 0);
           cp_async_16(sbase + r * 128 + ((c ^ (r & 7)) << 4), p.kv + static_cast<int64_t>(prow) * kRowBytes + blk * 128 + c * 16);
         }
-        cp_async_mbar_arrive_noinc(&bar[B_KFULL + slot]);
+        cp_async_mbar_arrive_noinc(&bar[B_KFULL + blk]);
       }
       if (!ok) asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp == kMmaWarp) {
@@ -298,76 +319,77 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t idesc = umma_idesc(128, kTile, 1, 0, 0);
         const uint64_t kdesc0 = umma_desc_sw128(smem_u32(base + Smem::kKRing), 16, 1024);
+        const uint64_t rrdesc0 = umma_desc_sw128(smem_u32(base + Smem::kRRing), 16, 1024);
         const uint64_t rdesc = umma_desc_sw128(smem_u32(base + Smem::kQRope), 16, 1024);
         for (int i = 0; i < ntiles && ok; ++i) {
           const int sb = i & 1;
           ok = mbar_wait(&bar[B_SFREE + sb], ((i >> 1) & 1) ^ 1, p.status, kDevErrTimeout);
           if (!ok) break;
           const uint32_t d = tmem + kColS + kTile * sb;
-          for (int blk = 0; blk < 9; ++blk) {
-            const int u = i * 9 + blk, slot = u % kKSlots;
-            ok = mbar_wait(&bar[B_KFULL + slot], (u / kKSlots) & 1, p.status, kDevErrTimeout);
+          for (int blk = 0; blk < kKSlots && ok; ++blk) {  // latent dims 0..511: A = Q from TMEM
+            ok = mbar_wait(&bar[B_KFULL + blk], i & 1, p.status, kDevErrTimeout);
             if (!ok) break;
             fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tensor-core reads
             tc_fence_after();
-            const uint64_t bd = kdesc0 + static_cast<uint64_t>((slot * kBlk) >> 4);
-            if (blk < 8) {
+            const uint64_t bd = kdesc0 + static_cast<uint64_t>((blk * kBlk) >> 4);
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                mma_bf16_ts(d, tmem + kColQ + 32 * blk + 8 * kk, bd + 2 * kk, idesc, (blk | kk) ? 1u : 0u);
-            } else {
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ts(d, tmem + kColQ + 32 * blk + 8 * kk, bd + 2 * kk, idesc, (blk | kk) ? 1u : 0u);
+            mma_commit(&bar[B_KEMPTY + blk]);
+          }
+          if (!ok) break;
+          {  // rope dims 512..575: A = Q rope from shared memory
+            const int rs = i % kRSlots;
+            ok = mbar_wait(&bar[B_RFULL + rs], (i / kRSlots) & 1, p.status, kDevErrTimeout);
+            if (!ok) break;
+            tc_fence_after();
+            const uint64_t bd = rrdesc0 + static_cast<uint64_t>((rs * kBlk) >> 4);
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(d, rdesc + 2 * kk, bd + 2 * kk, idesc, 1u);
-            }
-            mma_commit(&bar[B_KEMPTY + slot]);
+            for (int kk = 0; kk < 4; ++kk) mma_bf16_ss(d, rdesc + 2 * kk, bd + 2 * kk, idesc, 1u);
+            mma_commit(&bar[B_REMPTY + rs]);
           }
           if (!ok) break;
           mma_commit(&bar[B_SFULL + sb]);
         }
       }
       __syncwarp();
-    } else if (warp == kCopyWarp) {
-      // ---------- S-CTA copier: staging -> the O-CTA's P buffer i & 1, one bulk copy per tile ----------
-      if (lane == 0 && ntiles > 0) {
-        const uint8_t* stage = base + Smem::kPStage;
-        const uint32_t peer_p = peer_addr(smem_u32(base + Smem::kP), 1);
-        const uint32_t peer_pfull = peer_addr(smem_u32(&bar[B_PFULL]), 1);
-        bool ok = true;
-        for (int i = 0; i < ntiles && ok; ++i) {
-          const int sb = i & 1;
-          // all eight softmax warps wrote block i, and the O-CTA's MMA of tile i - 2 released buffer sb
-          ok = mbar_wait(&bar[B_PSFULL], i & 1, p.status, kDevErrTimeout) &&
-               mbar_wait(&bar[B_PFREE + sb], ((i >> 1) & 1) ^ 1, p.status, kDevErrTimeout);
-          if (!ok) break;
-          mbar_arrive_expect_tx_remote(peer_pfull + static_cast<uint32_t>(sb * 8), kPShip);
-          bulk_copy_to_peer(peer_p + static_cast<uint32_t>(sb * kPStride), stage, kPShip,
-                            peer_pfull + static_cast<uint32_t>(sb * 8));
-          bulk_commit_group();
-          bulk_wait_read_all();  // the staging buffer may be rewritten
-          mbar_arrive(&bar[B_PSFREE]);
+    } else if (warp == kRopeWarp) {
+      // ---------- S-CTA rope producer: dims 512..575 of a tile's 128 rows, 32 TMA gathers of 4 rows ----------
+      // (the TMA engine runs beside the cp.async path and adds to the gather rate of this SM)
+      bool ok = true;
+      if (lane == 0 && ntiles > 0) tma_prefetch_desc(&kvmap);
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const int rs = i % kRSlots;
+        bool w = true;
+        if (lane == 0) {
+          w = mbar_wait(&bar[B_REMPTY + rs], ((i / kRSlots) & 1) ^ 1, p.status, kDevErrTimeout);
+          if (w) mbar_arrive_expect_tx(&bar[B_RFULL + rs], kBlk);
         }
-        // the O-CTA's last multicast commits land in this CTA's barriers: wait for them before exit
-        if (ok) {
-          const int i1 = ntiles - 1;
-          mbar_wait(&bar[B_PFREE + (i1 & 1)], (i1 >> 1) & 1, p.status, kDevErrTimeout);
-          if (ntiles > 1) mbar_wait(&bar[B_PFREE + ((i1 - 1) & 1)], ((i1 - 1) >> 1) & 1, p.status, kDevErrTimeout);
-        }
+        ok = __shfl_sync(0xffffffffu, w, 0);
+        if (!ok) break;
+        const int32_t* rr = rows + i * kTile + 4 * lane;
+        tma_gather4(base + Smem::kRRing + rs * kBlk + lane * 512, &kvmap, 512, max(rr[0], 0), max(rr[1], 0),
+                    max(rr[2], 0), max(rr[3], 0), &bar[B_RFULL + rs]);
       }
+      // no gather may still be landing when the CTA exits (the MMA normally consumed them all)
+      if (lane == 0 && ok)
+        for (int i = max(0, ntiles - kRSlots); i < ntiles; ++i)
+          mbar_wait(&bar[B_RFULL + i % kRSlots], (i / kRSlots) & 1, p.status, kDevErrTimeout);
       __syncwarp();
     } else {
       // ---------- S-CTA softmax (warps 21..28: thread = head h, keys 64*sub .. 64*sub+63) ----------
       float* red = reinterpret_cast<float*>(base + Smem::kRed);    // [2][kSubs][128]
       float* redl = reinterpret_cast<float*>(base + Smem::kRedL);  // [2][kSubs][128]: l, lr
-      uint8_t* stage = base + Smem::kPStage;
+      const uint32_t peer_p = peer_addr(smem_u32(base + Smem::kP), 1);
+      const uint32_t peer_pfull = peer_addr(smem_u32(&bar[B_PFULL]), 1);
       float m_ref = -INFINITY, l = 0.f, lr = 0.f;
       bool ok = true;
       if (ntiles > 0) {
-        // Q dims 0..511: blocks 4*sub .. 4*sub+3 (ring slots / PStage) -> TMEM columns (lane = head)
+        // Q dims 0..511: blocks 4*sub .. 4*sub+3 (ring slots) -> TMEM columns (lane = head)
         ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_QROPE], 0, p.status, kDevErrTimeout));
         if (ok) {
           for (int blk = 4 * sub; blk < 4 * sub + 4; ++blk) {
-            const uint8_t* rowp =
-                base + (blk < kKSlots ? Smem::kKRing + blk * kBlk : Smem::kPStage + (blk - kKSlots) * kBlk) + h * 128;
+            const uint8_t* rowp = base + Smem::kKRing + blk * kBlk + h * 128;
             uint32_t r[32];
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -419,13 +441,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           m_ref = tmax;
         }
         const bool quad_rescale = __any_sync(0xffffffffu, need && i > 0);
-        // the previous P block must have left the staging buffer
-        ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_PSFREE], (i & 1) ^ 1, p.status, kDevErrTimeout));
+        // the O-CTA's product of tile i - 2 must have released its P buffer sb
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_PFREE + sb], ((i >> 1) & 1) ^ 1, p.status, kDevErrTimeout));
         if (!ok) break;
-        // pass 2: P[h, 64*sub .. +63] (bf16) into the staging copy of the peer's K-major swizzled
-        // P buffer: block sub (64 keys), chunks of 8 keys XOR-swizzled by head
+        const uint32_t pbuf = peer_p + static_cast<uint32_t>(sb * kPStride);
+        const uint32_t pbar = peer_pfull + static_cast<uint32_t>(sb * 8);
+        // the one arrival of the peer's PFULL[sb] phase, with the bytes the st.async below deliver
+        if (warp == kSoftWarp0 && lane == 0) mbar_arrive_expect_tx_remote(pbar, kPShip);
+        // pass 2: P[h, 64*sub .. +63] (bf16) straight into the peer's K-major swizzled P buffer:
+        // block sub (64 keys), chunks of 8 keys XOR-swizzled by head
         const float m_use = (m_ref > -INFINITY) ? m_ref : 0.f;  // m_ref = -inf: every key so far masked
-        uint8_t* prow = stage + sub * kBlk + h * 128;
+        const uint32_t prow = pbuf + static_cast<uint32_t>(sub * kBlk + h * 128);
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
           uint32_t v[32];
@@ -445,19 +471,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               w[q2] = *reinterpret_cast<const uint32_t*>(&bp);
             }
             const int chunk = 4 * c + q8;  // chunk 0..7 within block `sub`
-            *reinterpret_cast<uint4*>(prow + (((chunk ^ (h & 7))) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+            st_async_v4(prow + static_cast<uint32_t>((chunk ^ (h & 7)) << 4), w[0], w[1], w[2], w[3], pbar);
           }
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[B_SFREE + sb]);
         if (sub == 0) {
-          reinterpret_cast<float*>(stage + kPAlpha)[h] = alpha;
-          if (lane == 0) reinterpret_cast<uint32_t*>(stage + kPFlags)[quad] = quad_rescale ? 1u : 0u;
+          st_async_b32(pbuf + static_cast<uint32_t>(kPAlpha + h * 4), __float_as_uint(alpha), pbar);
+          if (lane == 0) st_async_b32(pbuf + static_cast<uint32_t>(kPFlags + quad * 4), quad_rescale ? 1u : 0u, pbar);
         }
-        fence_proxy_async_smem();  // staging writes (generic proxy) -> bulk copy reads (async proxy)
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[B_PSFULL]);
       }
       // per-head sums over the quadrant's warps, then the final statistics (always sent, so the
       // O-CTA never waits in vain)
@@ -480,6 +503,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         st_cluster_f32(peer_stats + static_cast<uint32_t>((256 + h) * 4), lrt);
         mbar_arrive_remote(peer_addr(smem_u32(&bar[B_STATS]), 1));
       }
+      // the O-CTA's last multicast commits land in this CTA's barriers: wait for them before exit
+      if (ok && ntiles > 0 && warp == kSoftWarp0 && lane == 0) {
+        const int i1 = ntiles - 1;
+        mbar_wait(&bar[B_PFREE + (i1 & 1)], (i1 >> 1) & 1, p.status, kDevErrTimeout);
+        if (ntiles > 1) mbar_wait(&bar[B_PFREE + ((i1 - 1) & 1)], ((i1 - 1) >> 1) & 1, p.status, kDevErrTimeout);
+      }
+      __syncwarp();
     }
   } else {
     if (warp < kProdWarps) {
@@ -515,6 +545,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           ok = mbar_wait(&bar[B_OREADY + pb], (i >> 1) & 1, p.status, kDevErrTimeout) &&
                mbar_wait_cluster(&bar[B_PFULL + pb], (i >> 1) & 1, p.status, kDevErrTimeout);
           if (!ok) break;
+          fence_proxy_async_smem();  // P arrived by st.async -> tensor-core reads
           tc_fence_after();
           const uint64_t pd = pdesc0 + static_cast<uint64_t>((pb * kPStride) >> 4);
           for (int qd = 0; qd < 4; ++qd) {
@@ -539,7 +570,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
       __syncwarp();
-    } else if (warp < kCopyWarp) {
+    } else if (warp < kSoftWarp0 + kSoftWarps) {
       // ---------- O-CTA correction + epilogue (warps 21..28: head h, O columns 256*sub .. +255) ------
       const volatile float* stats = reinterpret_cast<const volatile float*>(base + Smem::kStats);
       const uint32_t ocol = tmem + lane_base + kColO + 256 * sub;
@@ -581,7 +612,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const float inv = (have_o && lr > 0.f) ? 1.f / lr : 0.f;
       const float lse_nat = (have_o && l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
       if (p.nsplit == 1) {
-        uint16_t* dst = p.out + (static_cast<int64_t>(t) * H + h) * kDV + 256 * sub;
+        // normalised bf16 O -> the V ring (idle once every P V product has completed) as 8 boxes of
+        // [H heads][64 dims], 128-byte swizzled; one thread writes the boxes out with TMA stores
+        uint8_t* ost = base + Smem::kVRing;
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
           uint32_t o[32];
@@ -592,7 +625,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 32; ++j) o[j] = 0u;
           }
           if (h < H) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+            uint8_t* rowp = ost + (4 * sub + (c >> 1)) * kBlk + h * 128;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               uint4 w;
@@ -600,11 +633,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               w.y = pack_bf16x2(__uint_as_float(o[8 * j + 2]) * inv, __uint_as_float(o[8 * j + 3]) * inv);
               w.z = pack_bf16x2(__uint_as_float(o[8 * j + 4]) * inv, __uint_as_float(o[8 * j + 5]) * inv);
               w.w = pack_bf16x2(__uint_as_float(o[8 * j + 6]) * inv, __uint_as_float(o[8 * j + 7]) * inv);
-              d4[j] = w;
+              const int chunk = 4 * (c & 1) + j;
+              *reinterpret_cast<uint4*>(rowp + ((chunk ^ (h & 7)) << 4)) = w;
             }
           }
         }
         if (sub == 0 && h < H && p.lse) p.lse[static_cast<int64_t>(t) * H + h] = lse_nat;
+        fence_proxy_async_smem();  // staging writes (generic proxy) -> TMA store reads (async proxy)
+        named_bar_sync(1, 32 * kSoftWarps);
+        if (warp == kSoftWarp0 && lane == 0) {
+          for (int box = 0; box < 8; ++box) tma_store_3d(&omap, ost + box * kBlk, 64 * box, 0, t);
+          bulk_commit_group();
+          bulk_wait_all();
+        }
       } else {
         const int64_t prow = (static_cast<int64_t>(t) * p.nsplit + split) * H + h;
         float* dst = p.part_o + prow * kDV + 256 * sub;
@@ -730,15 +771,26 @@ int launch_sparse_mla(const BatchDev& b, const void* plan, const void* q, int H,
   }
   prm.status = &pv.hdr->status;
 
-  CUtensorMap qmap;
+  CUtensorMap qmap, kvmap, omap;
   int e = make_tmap_2d(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, kDLat, static_cast<uint64_t>(b.T) * H,
                        kDLat * 2, 64, 128);
   if (e) return e;
+  // latent rows, one row high boxes of 64 dims (TMA gather of the rope block)
+  e = make_tmap_2d(&kvmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kv_cache, kDLat,
+                   static_cast<uint64_t>(b.num_pages) * kPage, kDLat * 2, 64, 1);
+  if (e) return e;
+  memset(&omap, 0, sizeof(omap));
+  if (prm.nsplit == 1) {  // out [T][H][512] bf16, boxes of 64 dims x H heads of one row
+    e = make_tmap_3d(&omap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, out, kDV, static_cast<uint64_t>(H),
+                     static_cast<uint64_t>(b.T), kDV * 2, static_cast<uint64_t>(H) * kDV * 2, 64,
+                     static_cast<uint32_t>(H), 1);
+    if (e) return e;
+  }
   cudaError_t ce =
       cudaFuncSetAttribute(sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem::kDynamic);
   if (ce != cudaSuccess) return static_cast<int>(ce);
   dim3 grid(2 * b.T * prm.nsplit, 1, 1);
-  sparse_mla_kernel<<<grid, kThreads, Smem::kDynamic, static_cast<cudaStream_t>(stream)>>>(qmap, prm);
+  sparse_mla_kernel<<<grid, kThreads, Smem::kDynamic, static_cast<cudaStream_t>(stream)>>>(qmap, kvmap, omap, prm);
   ce = cudaGetLastError();
   if (ce != cudaSuccess) return static_cast<int>(ce);
   if (prm.nsplit > 1) {

@@ -3,14 +3,23 @@
 // formula; when the prefix holds no more than k positions all of them are taken, the handbook's
 // k = min(L, TOPK) in "MTP 与稀疏注意力：NSA 与 DSA", section "稀疏注意力：NSA 与 DSA").
 //
-// One CTA of 1024 threads per query row. Scores become order-preserving uint32 keys; a radix
-// select over 11 + 11 + 10 bits finds the exact k-th largest key with shared-memory histograms
-// (warp-aggregated atomics: scores crowd into a few exponent bins). A last pass over contiguous
-// per-warp segments (ballot-ordered, two block scans) emits every position above the threshold and
-// the first `remaining` positions equal to it, in increasing position order, so the result is
-// deterministic: among equal scores the smaller position wins.
-// Rows up to kCacheCap scores are kept in shared memory after the first read; longer rows are
-// re-read from L2 on each pass.
+// One CTA of 1024 threads per query row; L = p + 1 visible scores.
+//  1. Scores become order-preserving uint32 keys (one float4 per thread per chunk of 4096
+//     positions, all loads in flight); the row's smallest and largest key bound the search.
+//  2. A 2048-bin histogram linear in the score value between the row's minimum and maximum
+//     (floating-point subtraction and scaling are monotonic, so bins stay ordered) locates the bin
+//     holding the k-th largest score; real score rows spread over many bins, so plain shared-memory
+//     atomics rarely collide and the boundary bin holds a handful of keys. Rows this cannot split
+//     (infinities, NaN, heavy ties, an overfull boundary bin) narrow further in key space: bins
+//     (key - lo) >> s over the bin's exact key interval [lo, lo + W), s the smallest shift that
+//     fits W into 2048 bins, until the boundary bin is small or a single key value.
+//  3. Once that bin holds at most kCandCap keys, they are copied out and the k-th largest key
+//     theta is found exactly by counting, for each candidate, the candidates at least as large.
+//  4. Emission in increasing position order: every key above theta, then the first
+//     `ties` keys equal to theta (equal scores: the smaller position wins), so the result is
+//     deterministic. Per-(chunk, warp) counts and one warp-level scan give each warp its offsets.
+// Rows of up to kCacheCap keys keep their keys in shared memory; longer rows re-read the scores
+// (L2-resident: the indexer just wrote them) in each pass.
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -24,21 +33,21 @@ namespace {
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
-constexpr int kCacheCap = 24576;  // 96 KB of keys in shared memory
+constexpr int kChunk = 4 * kThreads;  // positions per chunk (one float4 per thread)
+constexpr int kCacheCap = 32768;      // keys kept in shared memory (128 KB)
+constexpr int kCandCap = 128;         // candidates resolved by counting
+constexpr int kGroup = 4;             // chunks whose loads are in flight together
+constexpr int kMaxChunks = kMaxTopKRow / kChunk;  // 64 chunks: rows up to 262144 positions
+static_assert(kMaxChunks % kGroup == 0, "chunk groups");
+static_assert(kCandCap <= kThreads, "one candidate per thread");
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t b = __float_as_uint(f);
   if (b == 0x80000000u) b = 0u;  // -0 ranks as +0
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
-
-// hist[bin] += 1 for every lane, one atomic per distinct bin in the warp (scores cluster in a
-// few exponent bins, so plain per-lane atomics would serialise on them).
-__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active) {
-  const uint32_t act = __ballot_sync(0xffffffffu, active);
-  if (!active) return;
-  const uint32_t peers = __match_any_sync(act, bin);
-  if ((threadIdx.x & 31) == static_cast<uint32_t>(__ffs(peers) - 1)) atomicAdd(&hist[bin], __popc(peers));
+__device__ __forceinline__ float key_value(uint32_t u) {  // inverse of order_key (-0 comes back as +0)
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
 }
 
 // Block-wide inclusive scan of one value per thread; `scratch` holds kWarps ints.
@@ -68,111 +77,344 @@ __device__ __forceinline__ int block_inclusive_scan(int v, int* scratch, int* to
   return r;
 }
 
+struct Keys4 {
+  uint32_t k[4];
+};
+
 __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restrict__ row_pos,
                                                         const float* __restrict__ scores, int64_t ld, int k,
-                                                        int32_t* __restrict__ S, int use_cache) {
-  extern __shared__ uint32_t tk_smem[];
-  uint32_t* hist = tk_smem;                // [kBins]
-  uint32_t* cache = tk_smem + kBins;       // [kCacheCap] when use_cache
+                                                        int32_t* __restrict__ S, int cache_cap) {
+  extern __shared__ __align__(16) uint32_t tk_smem[];
+  uint32_t* hist = tk_smem;                 // [kBins]
+  uint32_t* cand = tk_smem + kBins;         // [kCandCap]
+  uint32_t* cache = cand + kCandCap;        // [cache_cap]
   __shared__ int scan_scratch[kWarps];
-  __shared__ uint32_t sh_prefix, sh_remaining;
+  __shared__ uint32_t red_min[kWarps], red_max[kWarps];
+  __shared__ uint32_t sh_lo, sh_remaining, sh_ncand, sh_done;
+  __shared__ int2 cnt[kMaxChunks][kWarps];  // per (chunk, warp): (above theta, equal to theta)
 
   const int t = blockIdx.x;
   const int L = __ldg(row_pos + t) + 1;
   const float* row = scores + static_cast<int64_t>(t) * ld;
   int32_t* out = S + static_cast<int64_t>(t) * k;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
 
   if (L <= k) {
-    for (int j = threadIdx.x; j < k; j += kThreads) out[j] = (j < L) ? j : -1;
+    for (int j = tid; j < k; j += kThreads) out[j] = (j < L) ? j : -1;
     return;
   }
-  const bool cached = use_cache && L <= kCacheCap;
+  const bool cached = L <= cache_cap;
+  const int nchunks = (L + kChunk - 1) / kChunk;
 
-  uint32_t prefix = 0, mask = 0, remaining = static_cast<uint32_t>(k);
-  const int shifts[3] = {21, 10, 0};
-  const int widths[3] = {11, 11, 10};
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = shifts[pass];
-    const uint32_t nb = 1u << widths[pass];
-    const uint32_t bmask = nb - 1u;
-    for (uint32_t i = threadIdx.x; i < kBins; i += kThreads) hist[i] = 0u;
-    __syncthreads();
-    const int L_pad = (L + 31) & ~31;  // whole warps take part in the aggregated atomics
-    if (pass == 0) {
-      for (int j = threadIdx.x; j < L_pad; j += kThreads) {
-        uint32_t u = 0;
-        if (j < L) {
-          u = order_key(__ldg(row + j));
-          if (cached) cache[j] = u;
+  // keys of this thread in chunks cg .. cg + kGroup - 1 (all loads issued before any is used);
+  // positions >= L report nv = 0 and key 0
+  auto load_group = [&](int cg, Keys4 (&r)[kGroup], int (&nv)[kGroup]) {
+    float4 f[kGroup];
+#pragma unroll
+    for (int g = 0; g < kGroup; ++g) {
+      const int j0 = (cg + g) * kChunk + 4 * tid;
+      nv[g] = max(0, min(4, L - j0));
+      if (nv[g] > 0) {
+        if (cached) {
+          const uint4 v = *reinterpret_cast<const uint4*>(cache + j0);
+          r[g].k[0] = v.x, r[g].k[1] = v.y, r[g].k[2] = v.z, r[g].k[3] = v.w;
+        } else {
+          f[g] = __ldg(reinterpret_cast<const float4*>(row + j0));  // j0 + 3 < ld: ld % 4 == 0
         }
-        hist_add(hist, u >> shift, j < L);
       }
-    } else {
-      for (int j = threadIdx.x; j < L_pad; j += kThreads) {
-        uint32_t u = 0;
-        if (j < L) u = cached ? cache[j] : order_key(__ldg(row + j));
-        hist_add(hist, (u >> shift) & bmask, j < L && (u & mask) == prefix);
+    }
+#pragma unroll
+    for (int g = 0; g < kGroup; ++g) {
+      if (nv[g] == 0) {
+        r[g].k[0] = r[g].k[1] = r[g].k[2] = r[g].k[3] = 0u;
+      } else if (!cached) {
+        r[g].k[0] = order_key(f[g].x), r[g].k[1] = order_key(f[g].y);
+        r[g].k[2] = order_key(f[g].z), r[g].k[3] = order_key(f[g].w);
+      }
+    }
+  };
+
+  // ---- 1. keys, row minimum and maximum ----
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  for (int cg = 0; cg < nchunks; cg += kGroup) {
+    float4 f[kGroup];
+    int nv[kGroup];
+#pragma unroll
+    for (int g = 0; g < kGroup; ++g) {
+      const int j0 = (cg + g) * kChunk + 4 * tid;
+      nv[g] = max(0, min(4, L - j0));
+      if (nv[g] > 0) f[g] = __ldg(reinterpret_cast<const float4*>(row + j0));
+    }
+#pragma unroll
+    for (int g = 0; g < kGroup; ++g) {
+      if (nv[g] == 0) continue;
+      const uint32_t u[4] = {order_key(f[g].x), order_key(f[g].y), order_key(f[g].z), order_key(f[g].w)};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (e < nv[g]) kmin = min(kmin, u[e]), kmax = max(kmax, u[e]);
+      if (cached)
+        *reinterpret_cast<uint4*>(cache + (cg + g) * kChunk + 4 * tid) = make_uint4(u[0], u[1], u[2], u[3]);
+    }
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if (lane == 0) red_min[wid] = kmin, red_max[wid] = kmax;
+  for (int i = tid; i < kBins; i += kThreads) hist[i] = 0u;
+  __syncthreads();
+  kmin = __reduce_min_sync(0xffffffffu, red_min[lane]);
+  kmax = __reduce_max_sync(0xffffffffu, red_max[lane]);
+
+  uint32_t lo = kmin, wmax = kmax - kmin;  // key-space range [lo, lo + wmax]
+  uint32_t remaining = static_cast<uint32_t>(k);
+  uint32_t theta = kmax;
+  bool found = false;
+
+  // theta = the largest candidate value v with #(candidates >= v) >= remaining; on return
+  // `remaining` counts the keys equal to theta that are taken. cand[0 .. ncand) holds the keys.
+  auto resolve_candidates = [&](uint32_t ncand) {
+    uint32_t best = 0u;
+    bool have = false;
+    if (static_cast<uint32_t>(tid) < ncand) {
+      const uint32_t v = cand[tid];
+      uint32_t ge = 0;
+      for (uint32_t j = 0; j < ncand; ++j) ge += (cand[j] >= v) ? 1u : 0u;
+      if (ge >= remaining) best = v, have = true;
+    }
+    best = __reduce_max_sync(0xffffffffu, have ? best : 0u);
+    if (lane == 0) red_max[wid] = best;
+    __syncthreads();
+    theta = __reduce_max_sync(0xffffffffu, red_max[lane]);
+    const uint32_t v = (static_cast<uint32_t>(tid) < ncand) ? cand[tid] : 0u;
+    const int gt = __syncthreads_count(static_cast<uint32_t>(tid) < ncand && v > theta);
+    remaining -= static_cast<uint32_t>(gt);
+  };
+  // copies the keys satisfying `pred` into cand (their number is known to be <= kCandCap)
+  auto compact = [&](auto pred) {
+    for (int cg = 0; cg < nchunks; cg += kGroup) {
+      Keys4 r[kGroup];
+      int nv[kGroup];
+      load_group(cg, r, nv);
+#pragma unroll
+      for (int g = 0; g < kGroup; ++g) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const bool in = e < nv[g] && pred(r[g].k[e]);
+          const uint32_t act = __ballot_sync(0xffffffffu, in);
+          if (act == 0u) continue;
+          const int first = __ffs(act) - 1;
+          uint32_t base = 0;
+          if (lane == first) base = atomicAdd(&sh_done, static_cast<uint32_t>(__popc(act)));
+          base = __shfl_sync(0xffffffffu, base, first);
+          if (in) cand[base + __popc(act & ((1u << lane) - 1u))] = r[g].k[e];
+        }
       }
     }
     __syncthreads();
-    // counts from the top bin down: thread i owns descending bins 2i, 2i+1
-    const int d0 = 2 * threadIdx.x, d1 = d0 + 1;
+  };
+  // hist[bin(key)] += 1 over the keys with bin(key) < kBins (one atomic per warp when all agree)
+  auto histogram = [&](auto bin_of) {
+    for (int cg = 0; cg < nchunks; cg += kGroup) {
+      Keys4 r[kGroup];
+      int nv[kGroup];
+      load_group(cg, r, nv);
+#pragma unroll
+      for (int g = 0; g < kGroup; ++g) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t bin = e < nv[g] ? bin_of(r[g].k[e]) : 0xffffffffu;
+          const bool in = bin < static_cast<uint32_t>(kBins);
+          const uint32_t act = __ballot_sync(0xffffffffu, in);
+          if (act == 0u) continue;
+          const int first = __ffs(act) - 1;
+          const uint32_t b0 = __shfl_sync(0xffffffffu, bin, first);
+          if (__all_sync(0xffffffffu, !in || bin == b0)) {
+            if (lane == first) atomicAdd(&hist[b0], static_cast<uint32_t>(__popc(act)));
+          } else if (in) {
+            atomicAdd(&hist[bin], 1u);
+          }
+        }
+      }
+    }
+    __syncthreads();
+  };
+  // the bin b (of nb, counted from the top) holding the remaining-th largest key:
+  // sh_bin = b, sh_remaining = remaining - (keys in higher bins), sh_ncand = keys in b
+  auto find_bin = [&](uint32_t nb) {
+    const int d0 = 2 * tid, d1 = d0 + 1;  // thread i owns descending bins 2i, 2i+1
     const uint32_t c0 = (static_cast<uint32_t>(d0) < nb) ? hist[nb - 1 - d0] : 0u;
     const uint32_t c1 = (static_cast<uint32_t>(d1) < nb) ? hist[nb - 1 - d1] : 0u;
     int total;
     const int incl = block_inclusive_scan(static_cast<int>(c0 + c1), scan_scratch, &total);
-    const uint32_t before = static_cast<uint32_t>(incl) - c0 - c1;  // count in bins above d0
+    const uint32_t before = static_cast<uint32_t>(incl) - c0 - c1;
     if (before < remaining && remaining <= before + c0) {
-      sh_prefix = prefix | ((nb - 1 - d0) << shift);
+      sh_lo = nb - 1 - d0;
       sh_remaining = remaining - before;
+      sh_ncand = c0;
     } else if (before + c0 < remaining && remaining <= before + c0 + c1) {
-      sh_prefix = prefix | ((nb - 1 - d1) << shift);
+      sh_lo = nb - 1 - d1;
       sh_remaining = remaining - before - c0;
+      sh_ncand = c1;
     }
+    if (tid == 0) sh_done = 0u;
     __syncthreads();
-    prefix = sh_prefix;
-    remaining = sh_remaining;
-    mask |= bmask << shift;
-    __syncthreads();
+  };
+
+  // ---- 2. value-linear first pass ----
+  {
+    const float fmin = key_value(kmin), fmax = key_value(kmax);
+    const float range = fmax - fmin;
+    const float vscale = static_cast<float>(kBins) / range;
+    if (isfinite(fmin) && isfinite(fmax) && isfinite(range) && range > 0.f && isfinite(vscale)) {
+      auto vbin = [&](uint32_t u) -> uint32_t {
+        const int b = static_cast<int>((key_value(u) - fmin) * vscale);  // >= 0: key >= kmin
+        return static_cast<uint32_t>(min(b, kBins - 1));
+      };
+      histogram(vbin);
+      find_bin(kBins);
+      const uint32_t bstar = sh_lo, ncand = sh_ncand;
+      remaining = sh_remaining;
+      if (ncand <= static_cast<uint32_t>(kCandCap)) {
+        compact([&](uint32_t u) { return vbin(u) == bstar; });
+        resolve_candidates(ncand);
+        found = true;
+      } else {
+        // the boundary bin is a contiguous key interval: narrow it in key space
+        uint32_t bmin = 0xffffffffu, bmax = 0u;
+        for (int cg = 0; cg < nchunks; cg += kGroup) {
+          Keys4 r[kGroup];
+          int nv[kGroup];
+          load_group(cg, r, nv);
+#pragma unroll
+          for (int g = 0; g < kGroup; ++g)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (e < nv[g] && vbin(r[g].k[e]) == bstar) bmin = min(bmin, r[g].k[e]), bmax = max(bmax, r[g].k[e]);
+        }
+        bmin = __reduce_min_sync(0xffffffffu, bmin);
+        bmax = __reduce_max_sync(0xffffffffu, bmax);
+        if (lane == 0) red_min[wid] = bmin, red_max[wid] = bmax;
+        for (int i = tid; i < kBins; i += kThreads) hist[i] = 0u;
+        __syncthreads();
+        lo = __reduce_min_sync(0xffffffffu, red_min[lane]);
+        wmax = __reduce_max_sync(0xffffffffu, red_max[lane]) - lo;
+        kmax = lo + wmax;
+        __syncthreads();  // red_min / red_max are reused below
+        if (wmax == 0u) {
+          theta = lo;
+          found = true;
+        }
+      }
+    }
   }
 
-  // Ordered emission. Warp w owns the contiguous positions [w*SEG, (w+1)*SEG), visited 32
-  // consecutive positions at a time (conflict-free, ballot-ordered). Two block scans over the
-  // per-warp counts rank the ties (the first `remaining` in position order are taken) and give
-  // each warp its output offset.
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  const int SEG = 32 * ((L + kThreads - 1) / kThreads);
-  const int wj0 = min(L, wid * SEG), wj1 = min(L, wj0 + SEG);
-  int w_gt = 0, w_tie = 0;
-  for (int base = wj0; base < wj1; base += 32) {
-    const int j = base + lane;
-    const uint32_t u = (j < wj1) ? (cached ? cache[j] : order_key(__ldg(row + j))) : 0u;
-    w_gt += __popc(__ballot_sync(0xffffffffu, j < wj1 && u > prefix));
-    w_tie += __popc(__ballot_sync(0xffffffffu, j < wj1 && u == prefix));
-  }
-  int total;
-  const int tie_incl = __shfl_sync(0xffffffffu, block_inclusive_scan(lane == 0 ? w_tie : 0, scan_scratch, &total), 0);
-  const int tie_take = max(0, min(w_tie, static_cast<int>(remaining) - (tie_incl - w_tie)));
-  const int sel = w_gt + tie_take;
-  const int sel_incl = __shfl_sync(0xffffffffu, block_inclusive_scan(lane == 0 ? sel : 0, scan_scratch, &total), 0);
-  int slot = sel_incl - sel, ties_left = tie_take;
-  for (int base = wj0; base < wj1; base += 32) {
-    const int j = base + lane;
-    const uint32_t u = (j < wj1) ? (cached ? cache[j] : order_key(__ldg(row + j))) : 0u;
-    const bool gt = j < wj1 && u > prefix;
-    const bool tie = j < wj1 && u == prefix;
-    const uint32_t tie_mask = __ballot_sync(0xffffffffu, tie);
-    const bool take = gt || (tie && __popc(tie_mask & lt_mask) < ties_left);
-    const uint32_t take_mask = __ballot_sync(0xffffffffu, take);
-    if (take) {
-      const int o = slot + __popc(take_mask & lt_mask);
-      if (o < k) out[o] = j;
+  // ---- 3. key-space narrowing of [lo, lo + wmax] down to the k-th largest key theta ----
+  for (int pass = 0; pass < 4 && !found; ++pass) {
+    int s = 0;
+    while ((wmax >> s) >= static_cast<uint32_t>(kBins)) ++s;
+    histogram([&](uint32_t u) -> uint32_t {
+      const uint32_t d = u - lo;
+      return d <= wmax ? (d >> s) : 0xffffffffu;
+    });
+    find_bin((wmax >> s) + 1u);
+    lo = lo + (sh_lo << s);
+    remaining = sh_remaining;
+    const uint32_t ncand = sh_ncand;
+    // the new range is bin b* of this pass, clipped to the largest key
+    wmax = min((1u << s) - 1u, kmax - lo);
+    if (s == 0 || wmax == 0) {  // one key value left: theta found
+      theta = lo;
+      found = true;
+      break;
     }
-    slot += __popc(take_mask);
-    ties_left -= min(__popc(tie_mask), ties_left);
+    if (ncand <= static_cast<uint32_t>(kCandCap)) {
+      const uint32_t clo = lo, cw = wmax;
+      compact([&](uint32_t u) { return (u - clo) <= cw; });
+      resolve_candidates(ncand);
+      found = true;
+      break;
+    }
+    for (int i = tid; i < kBins; i += kThreads) hist[i] = 0u;
+    __syncthreads();
   }
-  for (int s2 = total + static_cast<int>(threadIdx.x); s2 < k; s2 += kThreads) out[s2] = -1;
+  // theta: the k-th largest key; remaining: how many keys equal to theta are taken
+
+  // ---- 4. ordered emission ----
+  for (int cg = 0; cg < nchunks; cg += kGroup) {
+    Keys4 r[kGroup];
+    int nv[kGroup];
+    load_group(cg, r, nv);
+#pragma unroll
+    for (int g = 0; g < kGroup; ++g) {
+      int gt = 0, eq = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        gt += (e < nv[g] && r[g].k[e] > theta) ? 1 : 0;
+        eq += (e < nv[g] && r[g].k[e] == theta) ? 1 : 0;
+      }
+      gt = __reduce_add_sync(0xffffffffu, gt);
+      eq = __reduce_add_sync(0xffffffffu, eq);
+      if (lane == 0 && cg + g < nchunks) cnt[cg + g][wid] = make_int2(gt, eq);
+    }
+  }
+  __syncthreads();
+  if (wid == 0) {  // exclusive prefix over (chunk, warp) in position order
+    int2 carry = make_int2(0, 0);
+    for (int c = 0; c < nchunks; ++c) {
+      const int2 v = cnt[c][lane];
+      int2 x = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int yx = __shfl_up_sync(0xffffffffu, x.x, o), yy = __shfl_up_sync(0xffffffffu, x.y, o);
+        if (lane >= o) x.x += yx, x.y += yy;
+      }
+      cnt[c][lane] = make_int2(carry.x + x.x - v.x, carry.y + x.y - v.y);
+      carry.x += __shfl_sync(0xffffffffu, x.x, 31);
+      carry.y += __shfl_sync(0xffffffffu, x.y, 31);
+    }
+  }
+  __syncthreads();
+  const int ties = static_cast<int>(remaining);
+  for (int cg = 0; cg < nchunks; cg += kGroup) {
+    Keys4 r[kGroup];
+    int nv[kGroup];
+    load_group(cg, r, nv);
+#pragma unroll
+    for (int g = 0; g < kGroup; ++g) {
+      const int c = cg + g;
+      int gt = 0, eq = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        gt += (e < nv[g] && r[g].k[e] > theta) ? 1 : 0;
+        eq += (e < nv[g] && r[g].k[e] == theta) ? 1 : 0;
+      }
+      if (!__any_sync(0xffffffffu, gt + eq > 0)) continue;
+      // exclusive prefix of (gt, eq) over the lanes below, packed into one word (each <= 128)
+      const int packed = (eq << 16) | gt;
+      int x = packed;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      x -= packed;
+      const int2 base = cnt[c][wid];  // c < nchunks: a chunk past the row has no selected key
+      int gt_before = base.x + (x & 0xffff);
+      int eq_before = base.y + (x >> 16);
+      const int j0 = c * kChunk + 4 * tid;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (e >= nv[g]) break;
+        const uint32_t u = r[g].k[e];
+        if (u > theta) {
+          out[gt_before + min(eq_before, ties)] = j0 + e;
+          ++gt_before;
+        } else if (u == theta) {
+          if (eq_before < ties) out[gt_before + eq_before] = j0 + e;
+          ++eq_before;
+        }
+      }
+    }
+  }
 }
 
 }  // namespace
@@ -180,15 +422,14 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
 int launch_topk(const BatchDev& b, const void* plan, const float* scores, int64_t ld, int k, int32_t* S,
                 void* stream) {
   if (b.T == 0) return 0;
+  if (b.max_seq_len > kMaxChunks * kChunk) return static_cast<int>(cudaErrorInvalidValue);
   PlanView pv = plan_view(const_cast<void*>(plan), b.B, b.T);
-  const int use_cache = 1;
-  const int cap = b.max_seq_len < kCacheCap ? b.max_seq_len : kCacheCap;
-  const size_t smem = sizeof(uint32_t) * (kBins + static_cast<size_t>(cap));
+  const int cap = b.max_seq_len <= kCacheCap ? ((b.max_seq_len + 3) & ~3) : 0;
+  const size_t smem = sizeof(uint32_t) * (kBins + kCandCap + static_cast<size_t>(cap));
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(sizeof(uint32_t) * (kBins + kCacheCap)));
+                                       static_cast<int>(sizeof(uint32_t) * (kBins + kCandCap + kCacheCap)));
   if (e != cudaSuccess) return static_cast<int>(e);
-  topk_kernel<<<b.T, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(pv.row_pos, scores, ld, k, S,
-                                                                          use_cache && cap >= 1);
+  topk_kernel<<<b.T, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(pv.row_pos, scores, ld, k, S, cap);
   return static_cast<int>(cudaGetLastError());
 }
 

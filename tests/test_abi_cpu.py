@@ -93,6 +93,10 @@ def test_topk_and_mla_validation(lib):
     assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE, 384, 0, FAKE, None) == 2
     assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE, 384, 5000, FAKE, None) == 2
     assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE, 100, 16, FAKE, None) == 1
+    assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE, 386, 16, FAKE, None) == 1      # ld % 4
+    assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE + 4, 384, 16, FAKE, None) == 1  # misaligned scores
+    long_rows = batch(max_seq_len=262145, max_pages=4097)
+    assert lib.dsa_topk(ctypes.byref(long_rows), FAKE, FAKE, 262148, 16, FAKE, None) == 2
     mla = lambda **kw: lib.dsa_sparse_mla(
         ctypes.byref(b), FAKE, kw.get("q", FAKE), kw.get("H", 128), FAKE, FAKE, kw.get("k", 2048),
         kw.get("scale", 0.07), FAKE, None, kw.get("ws", FAKE), kw.get("ws_bytes", 1 << 30), None)
