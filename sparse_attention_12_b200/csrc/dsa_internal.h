@@ -6,6 +6,10 @@
 #include "../../include/dsa.h"
 
 #if defined(__CUDACC__)
+#include <cuda_runtime.h>
+#endif
+
+#if defined(__CUDACC__)
 #define DSA_HD __host__ __device__
 #else
 #define DSA_HD
@@ -107,5 +111,27 @@ size_t sparse_mla_ws_bytes(int T, int H, int k);
 int sparse_mla_splits(int T, int k);
 int launch_sparse_mla(const BatchDev& b, const void* plan, const void* q, int H, const void* kv_cache,
                       const int32_t* S, int k, float softmax_scale, void* out, float* lse, void* ws, void* stream);
+
+#if defined(__CUDACC__)
+// Launches every kernel of the library with programmatic stream serialization: its CTAs may be
+// scheduled while the previous kernel in the stream finishes (once all of that kernel's CTAs have
+// started), run their set-up, and wait in griddepcontrol.wait before touching memory an earlier
+// kernel writes or reads. Each kernel calls pdl_wait() before its first such access.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, void* stream,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+#endif
 
 }  // namespace dsa

@@ -14,6 +14,12 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Programmatic dependent launch: let the next kernel in the stream start its CTAs early, and wait
+// until the previous kernel has completed and its memory is visible (a no-op when the kernel was
+// launched without the attribute).
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
 __device__ __forceinline__ uint32_t warp_id() { return threadIdx.x >> 5; }
 
@@ -62,25 +68,47 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that lets the hardware suspend the thread until the phase completes or kSuspendNs
+// passes, so waiting warps sleep instead of spinning on the barrier (and take no issue slots
+// from the warps sharing their scheduler).
+constexpr uint32_t kSuspendNs = 1000000u;  // 1 ms
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase of `bar` with the given parity to complete. Gives up after ~kWaitLimitNs
 // (or as soon as another CTA reported an error), records `code` in the status word and
 // returns false. Every pipeline wait in this library goes through here.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
 static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint32_t* status, uint32_t code) {
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 255u) {
-      if (error_seen(status)) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        report_error(status, code);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_suspend(bar, parity)) return true;
+    if (error_seen(status)) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      report_error(status, code);
+      return false;
     }
   }
 }
+// Non-blocking test of a phase (the common case in pipelines that run ahead: already complete).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status, uint32_t code) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_test_wait(bar, parity)) return true;
   return mbar_wait_slow(bar, parity, status, code);
 }
 
@@ -95,17 +123,25 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
       : "memory");
   return ok != 0;
 }
+__device__ __forceinline__ bool mbar_try_wait_cluster_suspend(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
+      : "memory");
+  return ok != 0;
+}
 static __device__ __noinline__ bool mbar_wait_cluster_slow(uint64_t* bar, uint32_t parity, uint32_t* status,
                                                            uint32_t code) {
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((it & 255u) == 255u) {
-      if (error_seen(status)) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        report_error(status, code);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_cluster_suspend(bar, parity)) return true;
+    if (error_seen(status)) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      report_error(status, code);
+      return false;
     }
   }
 }

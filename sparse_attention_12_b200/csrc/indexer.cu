@@ -14,10 +14,12 @@
 // registers and writes one fp32 score per query; the per-head products never leave the SM.
 //
 // Persistent CTAs (one per SM) walk a contiguous slice of the plan's tile list. Warp roles:
-//   warp 0      TMA producer: key pages (via the block table) into a 6-stage ring, query tiles and
-//               the group's w / s^q into a 2-deep buffer
+//   warp 0      TMA producer: key pages (via the block table) into a ring of 9..12 stages, the
+//               tile's s^k into its own ring (cp.async), query tiles and the group's w / s^q into
+//               a 2-deep buffer
 //   warp 1      TMEM allocator and single-thread MMA issuer
-//   warps 2..9  epilogue (two warps per TMEM lane quadrant, splitting the group's queries)
+//   warps 2..9  epilogue (two warps per TMEM lane quadrant; the (tile, query) items alternate
+//               between the two, so a single-query decode group keeps both busy)
 // Decode tiles are HBM-bound (16 KB of keys per 128x64x128 MMA chain); prefill tiles are
 // tensor-bound with the 8 epilogue warps keeping pace with the MMA.
 #include <cuda.h>
@@ -31,9 +33,9 @@
 namespace dsa {
 namespace {
 
-constexpr int kStages = 6;
+constexpr int kMaxStages = 14;  // key stages: as many as shared memory holds next to the query buffers
+constexpr int kScaleSlots = 16;  // s^k of a tile (512 B) in its own ring: key stages free at MMA completion
 constexpr int kStageBytes = kIdxTileKeys * kDIdx;  // 16 KB
-constexpr int kQBufBytes = kIdxCols * kDIdx;       // 32 KB
 constexpr int kMaxAcc = 8;
 constexpr int kThreads = 320;
 constexpr int kEpiWarps = 8;
@@ -42,19 +44,20 @@ struct __align__(16) GroupMeta {
   int32_t row0, nq, pos0, req;
 };
 
+// Shared memory: the fixed part first, then two query buffers of qbytes (the group's query box,
+// 8 KB for one query of 64 heads, up to 32 KB) and as many 16 KB key stages as fit; the host
+// computes qbytes and the stage count (12 stages for decode, 9 for 256-row prefill groups).
 struct IdxSmem {
   // byte offsets relative to the 1024-aligned base
-  static constexpr int kStage0 = 0;
-  static constexpr int kQBuf0 = kStage0 + kStages * kStageBytes;  // 96 KB
-  static constexpr int kW = kQBuf0 + 2 * kQBufBytes;              // 160 KB: float [2][256]
-  static constexpr int kScale = kW + 2 * kIdxCols * 4;            // float [kStages][128]: s^k of the tile
-  static constexpr int kSq = kScale + kStages * kIdxTileKeys * 4; // float [2][16]
+  static constexpr int kW = 0;                                     // float [2][256]
+  static constexpr int kScale = kW + 2 * kIdxCols * 4;            // float [kScaleSlots][128]: s^k of a tile
+  static constexpr int kSq = kScale + kScaleSlots * kIdxTileKeys * 4;  // float [2][16]
   static constexpr int kMeta = kSq + 2 * 16 * 4;                  // GroupMeta [2]
   static constexpr int kBars = kMeta + 2 * 16;                    // uint64 barriers
-  static constexpr int kNumBars = 2 * kStages + 4 + 2 * kMaxAcc;
+  static constexpr int kNumBars = 2 * kMaxStages + 4 + 2 * kMaxAcc + 2 * kScaleSlots;
   static constexpr int kTmemSlot = kBars + kNumBars * 8;
-  static constexpr int kTotal = kTmemSlot + 16;
-  static constexpr int kDynamic = kTotal + 1024;  // slack for the manual 1024-byte alignment
+  static constexpr int kFixed = (kTmemSlot + 16 + 1023) / 1024 * 1024;  // query buffers start here
+  static constexpr int kLimit = 232448 - 1024;  // 227 KB less the slack for the 1024-byte alignment
 };
 
 struct IdxParams {
@@ -73,18 +76,31 @@ struct IdxParams {
   int ncols;      // TMEM columns per accumulator buffer (power of two >= 32)
   int nacc;       // accumulator buffers
   int qbox_rows;  // query rows per TMA box
+  int qbytes;     // bytes per query buffer (multiple of 1024)
+  int nstages;    // key stages
   uint32_t* status;
 };
 
-// Last group g with tile0[g] <= u.
-__device__ __forceinline__ int find_group(const int32_t* tile0, int G, int u) {
-  int lo = 0, hi = G;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(tile0 + mid) <= u)
-      lo = mid;
-    else
-      hi = mid - 1;
+// Last group g in [0, G) with tile0[g] <= u (tile0 strictly increasing, tile0[0] = 0 <= u),
+// searched by a whole warp with 32 probes per round: about log32(G) dependent loads.
+__device__ __forceinline__ int find_group_warp(const int32_t* tile0, int G, int u) {
+  const int lane = threadIdx.x & 31;
+  int lo = 0, hi = G - 1;  // the answer lies in [lo, hi]
+  while (hi > lo) {
+    const int span = hi - lo;
+    const int pos = lo + static_cast<int>((static_cast<int64_t>(lane + 1) * span + 31) / 32);  // in (lo, hi]
+    const bool le = __ldg(tile0 + pos) <= u;  // true on a prefix of the lanes
+    const uint32_t m = __ballot_sync(0xffffffffu, le);
+    const int l = m ? 31 - __clz(m) : -1;
+    const int p0 = __shfl_sync(0xffffffffu, pos, 0);
+    const int pl = __shfl_sync(0xffffffffu, pos, l < 0 ? 0 : l);
+    const int pn = __shfl_sync(0xffffffffu, pos, l < 31 ? l + 1 : 31);
+    if (l < 0) {
+      hi = p0 - 1;
+    } else {
+      lo = pl;
+      if (l < 31) hi = pn - 1;
+    }
   }
   return lo;
 }
@@ -102,27 +118,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   GroupMeta* g_meta = reinterpret_cast<GroupMeta*>(base + IdxSmem::kMeta);
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + IdxSmem::kBars);
   uint64_t* kfull = bars;
-  uint64_t* kempty = bars + kStages;
-  uint64_t* qfull = bars + 2 * kStages;
+  uint64_t* kempty = bars + kMaxStages;
+  uint64_t* qfull = bars + 2 * kMaxStages;
   uint64_t* qempty = qfull + 2;
   uint64_t* tfull = qempty + 2;
   uint64_t* tempty = tfull + kMaxAcc;
+  uint64_t* sfull = tempty + kMaxAcc;
+  uint64_t* sempty = sfull + kScaleSlots;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + IdxSmem::kTmemSlot);
 
   const int warp = warp_id(), lane = lane_id();
-  const int G = p.hdr->num_groups;
-  const int U = p.hdr->total_tiles;
-  const int u0 = static_cast<int>((static_cast<int64_t>(U) * blockIdx.x) / gridDim.x);
-  const int u1 = static_cast<int>((static_cast<int64_t>(U) * (blockIdx.x + 1)) / gridDim.x);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&kfull[s], 1);
-      mbar_init(&kempty[s], 1 + kEpiWarps);  // MMA done with the keys, epilogue with the scales
+    for (int s = 0; s < p.nstages; ++s) {
+      mbar_init(&kfull[s], 1);  // TMA bytes of the keys
+      mbar_init(&kempty[s], 1);  // MMA done with the keys
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&qfull[b], 1);
       mbar_init(&qempty[b], 1 + kEpiWarps);
+    }
+    for (int c = 0; c < kScaleSlots; ++c) {
+      mbar_init(&sfull[c], 32);          // one cp.async arrival per producer lane
+      mbar_init(&sempty[c], kEpiWarps);  // epilogue read the scales
     }
     for (int a = 0; a < kMaxAcc; ++a) {
       mbar_init(&tfull[a], 1);
@@ -138,6 +156,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&kmap);
     tma_prefetch_desc(&qmap);
   }
+  pdl_trigger();
+  pdl_wait();  // the plan, written by the previous kernel
+  const int G = p.hdr->num_groups;
+  const int U = p.hdr->total_tiles;
+  const int u0 = static_cast<int>((static_cast<int64_t>(U) * blockIdx.x) / gridDim.x);
+  const int u1 = static_cast<int>((static_cast<int64_t>(U) * (blockIdx.x + 1)) / gridDim.x);
+  const int g_first = (u0 < u1) ? find_group_warp(p.grp_tile0, G, u0) : 0;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -146,13 +171,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (u0 < u1) {
     if (warp == 0) {
       // ---------------- producer ----------------
-      int g = find_group(p.grp_tile0, G, u0);
+      int g = g_first;
       int gstart = __ldg(p.grp_tile0 + g), gend = __ldg(p.grp_tile0 + g + 1);
       GroupMeta gm{};
       int qcount = 0;
       int pg_base = -1;  // first logical page held in `pg_cache`
-      int pg_cache = 0;
+      int pg_cache = 0, pg_next = 0;  // this window's page ids and the next window's (prefetched)
       bool ok = true;
+      int s = 0, s_par = 1, c = 0, c_par = 1;  // ring positions of tile it and the parity to wait for
       for (int u = u0, it = 0; u < u1 && ok; ++u, ++it) {
         const bool newg = (u == u0) || (u == gend);
         if (u == gend) {
@@ -178,48 +204,55 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) {
             mbar_arrive_expect_tx(&qfull[qb], static_cast<uint32_t>(p.qbox_rows * kDIdx));
-            tma_load_2d(base + IdxSmem::kQBuf0 + qb * kQBufBytes, &qmap, 0, gm.row0 * NHI, &qfull[qb]);
+            tma_load_2d(base + IdxSmem::kFixed + qb * p.qbytes, &qmap, 0, gm.row0 * NHI, &qfull[qb]);
           }
           ++qcount;
           pg_base = -1;
         }
         const int kt = u - gstart;
         const int lp0 = 2 * kt;
-        // block-table window of 32 logical pages, refreshed every 16 tiles
+        // block-table window of 32 logical pages, refreshed every 16 tiles; the next window is
+        // loaded one window ahead so the refresh does not wait on memory
         if (pg_base < 0 || lp0 >= pg_base + 32) {
-          pg_base = lp0;
-          const int lp = pg_base + lane;
           const int npages = (gm.pos0 + gm.nq - 1) / kPage + 1;
-          pg_cache = (lp < npages) ? __ldg(p.bd.block_table + static_cast<int64_t>(gm.req) * p.bd.max_pages + lp) : 0;
+          const int32_t* bt = p.bd.block_table + static_cast<int64_t>(gm.req) * p.bd.max_pages;
+          if (pg_base >= 0 && lp0 == pg_base + 32) {
+            pg_cache = pg_next;
+          } else {
+            pg_cache = (lp0 + lane < npages) ? __ldg(bt + lp0 + lane) : 0;
+          }
+          pg_base = lp0;
+          pg_next = (pg_base + 32 + lane < npages) ? __ldg(bt + pg_base + 32 + lane) : 0;
         }
         const int pg0 = __shfl_sync(0xffffffffu, pg_cache, lp0 - pg_base);
         const int pg1 = __shfl_sync(0xffffffffu, pg_cache, lp0 + 1 - pg_base);
+        // every lane tests the two slots itself (no broadcast on the per-tile path)
+        ok = mbar_wait(&kempty[s], s_par, p.status, kDevErrTimeout) &&
+             mbar_wait(&sempty[c], c_par, p.status, kDevErrTimeout);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        const int p_last = gm.pos0 + gm.nq - 1;
+        const bool v1 = (lp0 + 1) * kPage <= p_last;
+        const int q0 = min(max(pg0, 0), p.bd.num_pages - 1), q1 = min(max(pg1, 0), p.bd.num_pages - 1);
         if (lane == 0) {
-          const int s = it % kStages;
-          ok = mbar_wait(&kempty[s], ((it / kStages) & 1) ^ 1, p.status, kDevErrTimeout);
-          if (ok) {
-            const int p_last = gm.pos0 + gm.nq - 1;
-            const bool v1 = (lp0 + 1) * kPage <= p_last;
-            if (pg0 < 0 || pg0 >= p.bd.num_pages || (v1 && (pg1 < 0 || pg1 >= p.bd.num_pages)))
-              report_error(p.status, kDevErrIndex);
-            uint8_t* dst = base + IdxSmem::kStage0 + s * kStageBytes;
-            float* sdst = g_scale + s * kIdxTileKeys;
-            const int q0 = min(max(pg0, 0), p.bd.num_pages - 1), q1 = min(max(pg1, 0), p.bd.num_pages - 1);
-            mbar_arrive_expect_tx(&kfull[s], static_cast<uint32_t>((v1 ? 2 : 1) * kPage * (kDIdx + 4)));
-            tma_load_2d(dst, &kmap, 0, pg0 * kPage, &kfull[s]);
-            bulk_load(sdst, p.kI_scale + static_cast<int64_t>(q0) * kPage, kPage * 4, &kfull[s]);
-            if (v1) {
-              tma_load_2d(dst + kPage * kDIdx, &kmap, 0, pg1 * kPage, &kfull[s]);
-              bulk_load(sdst + kPage, p.kI_scale + static_cast<int64_t>(q1) * kPage, kPage * 4, &kfull[s]);
-            }
-          }
+          if (pg0 < 0 || pg0 >= p.bd.num_pages || (v1 && (pg1 < 0 || pg1 >= p.bd.num_pages)))
+            report_error(p.status, kDevErrIndex);
+          uint8_t* dst = base + IdxSmem::kFixed + 2 * p.qbytes + s * kStageBytes;
+          mbar_arrive_expect_tx(&kfull[s], static_cast<uint32_t>((v1 ? 2 : 1) * kPage * kDIdx));
+          tma_load_2d(dst, &kmap, 0, q0 * kPage, &kfull[s]);
+          if (v1) tma_load_2d(dst + kPage * kDIdx, &kmap, 0, q1 * kPage, &kfull[s]);
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        // s^k of the tile's 128 keys: 16 bytes per lane (lanes 0..15 page 0, 16..31 page 1)
+        cp_async_16(smem_u32(g_scale + c * kIdxTileKeys + 4 * lane),
+                    p.kI_scale + static_cast<int64_t>(lane < 16 ? q0 : q1) * kPage + 4 * (lane & 15));
+        cp_async_mbar_arrive_noinc(&sfull[c]);
+        if (++s == p.nstages) s = 0, s_par ^= 1;
+        if (++c == kScaleSlots) c = 0, c_par ^= 1;
       }
+      asm volatile("cp.async.wait_all;" ::: "memory");
     } else if (warp == 1) {
       // ---------------- MMA issuer ----------------
       if (lane == 0) {
-        int g = find_group(p.grp_tile0, G, u0);
+        int g = g_first;
         int gend = __ldg(p.grp_tile0 + g + 1);
         int nq = 0, qcount = 0, qb = 0;
         bool ok = true;
@@ -236,15 +269,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             nq = __ldg(p.grp_nq + g);
             ++qcount;
           }
-          const int s = it % kStages;
+          const int s = it % p.nstages;
           const int a = it % p.nacc;
-          ok = mbar_wait(&kfull[s], (it / kStages) & 1, p.status, kDevErrTimeout) &&
+          ok = mbar_wait(&kfull[s], (it / p.nstages) & 1, p.status, kDevErrTimeout) &&
                mbar_wait(&tempty[a], ((it / p.nacc) & 1) ^ 1, p.status, kDevErrTimeout);
           if (!ok) break;
           tc_fence_after();
           const uint32_t idesc = umma_idesc(128, static_cast<uint32_t>(nq * NHI), 0, 0, 0);
-          const uint64_t ad = umma_desc_sw128(smem_u32(base + IdxSmem::kStage0 + s * kStageBytes), 16, 1024);
-          const uint64_t bd = umma_desc_sw128(smem_u32(base + IdxSmem::kQBuf0 + qb * kQBufBytes), 16, 1024);
+          const uint64_t ad =
+              umma_desc_sw128(smem_u32(base + IdxSmem::kFixed + 2 * p.qbytes + s * kStageBytes), 16, 1024);
+          const uint64_t bd = umma_desc_sw128(smem_u32(base + IdxSmem::kFixed + qb * p.qbytes), 16, 1024);
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * p.ncols);
 #pragma unroll
           for (int k = 0; k < kDIdx / 32; ++k)  // K step of 32 bytes = +2 in the start-address field
@@ -261,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int quad = warp & 3;
       const int half = ew >> 2;
       const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-      int g = find_group(p.grp_tile0, G, u0);
+      int g = g_first;
       int gstart = __ldg(p.grp_tile0 + g), gend = __ldg(p.grp_tile0 + g + 1);
       int qcount = 0, qb = 0;
       GroupMeta gm{};
@@ -283,33 +317,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kt = u - gstart;
         const int j = kt * kIdxTileKeys + quad * 32 + lane;
         const int p_last = gm.pos0 + gm.nq - 1;
-        const int s = it % kStages;
+        const int c = it % kScaleSlots;
         const int a = it % p.nacc;
-        ok = __all_sync(0xffffffffu, mbar_wait(&kfull[s], (it / kStages) & 1, p.status, kDevErrTimeout) &&
+        // (not kfull: key stages recycle at MMA completion and may run a whole ring ahead of here)
+        ok = __all_sync(0xffffffffu, mbar_wait(&sfull[c], (it / kScaleSlots) & 1, p.status, kDevErrTimeout) &&
                                          mbar_wait(&tfull[a], (it / p.nacc) & 1, p.status, kDevErrTimeout));
         if (!ok) break;
-        const float sk = (j <= p_last) ? g_scale[s * kIdxTileKeys + quad * 32 + lane] : 0.f;
+        const float sk = (j <= p_last) ? g_scale[c * kIdxTileKeys + quad * 32 + lane] : 0.f;
         tc_fence_after();
         const uint32_t t_row = tmem_base + lane_base + static_cast<uint32_t>(a * p.ncols);
-        for (int q = half; q < gm.nq; q += 2) {
-          const float* w = g_w + qb * kIdxCols + q * NHI;
-          float acc = 0.f;
+        // items (tile it, query q) alternate between the quadrant's two warps
+        for (int q = (half + it * gm.nq) & 1; q < gm.nq; q += 2) {
+          const float4* w4 = reinterpret_cast<const float4*>(g_w + qb * kIdxCols + q * NHI);
+          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;  // four chains: the head sum is latency-bound
+          auto accumulate = [&](const uint32_t* v, int nv, int w0) {
+#pragma unroll
+            for (int i = 0; i < nv / 4; ++i) {
+              const float4 ww = w4[w0 / 4 + i];
+              a0 = fmaf(ww.x, fmaxf(__uint_as_float(v[4 * i + 0]), 0.f), a0);
+              a1 = fmaf(ww.y, fmaxf(__uint_as_float(v[4 * i + 1]), 0.f), a1);
+              a2 = fmaf(ww.z, fmaxf(__uint_as_float(v[4 * i + 2]), 0.f), a2);
+              a3 = fmaf(ww.w, fmaxf(__uint_as_float(v[4 * i + 3]), 0.f), a3);
+            }
+          };
           if constexpr (NHI % 32 == 0) {
 #pragma unroll
             for (int c = 0; c < NHI / 32; ++c) {
               uint32_t v[32];
               tmem_ld32(t_row + static_cast<uint32_t>(q * NHI + c * 32), v);
               tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 32; ++i) acc = fmaf(w[c * 32 + i], fmaxf(__uint_as_float(v[i]), 0.f), acc);
+              accumulate(v, 32, c * 32);
             }
           } else {
             uint32_t v[16];
             tmem_ld16(t_row + static_cast<uint32_t>(q * NHI), v);
             tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) acc = fmaf(w[i], fmaxf(__uint_as_float(v[i]), 0.f), acc);
+            accumulate(v, 16, 0);
           }
+          const float acc = (a0 + a1) + (a2 + a3);
           float score = acc * g_sq[qb * 16 + q] * sk;
           if (j > gm.pos0 + q) score = -INFINITY;
           if (j < p.ld) p.scores[static_cast<int64_t>(gm.row0 + q) * p.ld + j] = score;
@@ -317,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&kempty[s]);
+          mbar_arrive(&sempty[c]);
           mbar_arrive(&tempty[a]);
           if (u + 1 == gend || u + 1 == u1) mbar_arrive(&qempty[qb]);
         }
@@ -424,10 +469,15 @@ static int launch_index_scores_t(const BatchDev& b, const void* plan, const uint
                    kDIdx, static_cast<uint32_t>(prm.qbox_rows));
   if (e) return e;
   auto kern = index_scores_kernel<NHI>;
-  cudaError_t ce = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, IdxSmem::kDynamic);
+  prm.qbytes = (prm.qbox_rows * kDIdx + 1023) / 1024 * 1024;
+  prm.nstages = (IdxSmem::kLimit - IdxSmem::kFixed - 2 * prm.qbytes) / kStageBytes;
+  if (prm.nstages > kMaxStages) prm.nstages = kMaxStages;
+  if (prm.nstages < 2) return static_cast<int>(cudaErrorInvalidValue);
+  const int smem = IdxSmem::kFixed + 2 * prm.qbytes + prm.nstages * kStageBytes + 1024;
+  cudaError_t ce = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (ce != cudaSuccess) return static_cast<int>(ce);
-  kern<<<num_sms(), kThreads, IdxSmem::kDynamic, static_cast<cudaStream_t>(stream)>>>(kmap, qmap, prm);
-  return static_cast<int>(cudaGetLastError());
+  return static_cast<int>(
+      launch_pdl(kern, dim3(num_sms()), dim3(kThreads), static_cast<size_t>(smem), stream, kmap, qmap, prm));
 }
 
 int launch_index_scores(const BatchDev& b, const void* plan, const uint8_t* qI, const float* qI_scale,

@@ -51,6 +51,8 @@ __device__ int32_t block_exclusive_scan(int32_t* data, int n, int32_t* warp_sums
   return carry;
 }
 
+constexpr int kPlanSmemMaxB = 3968;  // (3 B + 2) int32 stay under the 48 KB default
+
 // Last index i in [0, n) with a[i] <= key (a non-decreasing); -1 if none.
 __device__ __forceinline__ int upper_index(const int32_t* a, int n, int32_t key) {
   int lo = 0, hi = n;  // answer in [lo-1, hi-1]
@@ -64,46 +66,65 @@ __device__ __forceinline__ int upper_index(const int32_t* a, int n, int32_t key)
   return lo - 1;
 }
 
-__global__ void __launch_bounds__(kPlanThreads) plan_kernel(BatchDev bd, int nhI, void* plan_base) {
+// With B <= kPlanSmemMaxB the per-request arrays (cu_q, seq_lens, group offsets) are staged in
+// shared memory, so the per-row and per-group binary searches run there instead of through L2.
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(BatchDev bd, int nhI, void* plan_base, int staged) {
   __shared__ int32_t warp_sums[32];
+  extern __shared__ int32_t plan_smem[];  // [B+1] cu_q, [B] seq_lens, [B+1] group offsets when staged
   PlanView pv = plan_view(plan_base, bd.B, bd.T);
   const int B = bd.B, T = bd.T;
   const int qpg = kIdxCols / nhI;
   uint32_t* status = &pv.hdr->status;
+  pdl_trigger();
+  pdl_wait();  // the plan may still be read by the kernels of the previous call
+  const int32_t* cuq = bd.cu_q;
+  const int32_t* sl = bd.seq_lens;
+  int32_t* goff = pv.req_goff;
+  if (staged) {
+    int32_t* s_cuq = plan_smem;
+    int32_t* s_sl = plan_smem + (B + 1);
+    for (int i = threadIdx.x; i <= B; i += kPlanThreads) s_cuq[i] = __ldg(bd.cu_q + i);
+    for (int i = threadIdx.x; i < B; i += kPlanThreads) s_sl[i] = __ldg(bd.seq_lens + i);
+    cuq = s_cuq;
+    sl = s_sl;
+    goff = plan_smem + (2 * B + 1);
+  }
   if (threadIdx.x == 0) *status = 0u;
   __syncthreads();
 
   // groups per request, then their offsets
   for (int b = threadIdx.x; b < B; b += kPlanThreads) {
-    const int m = __ldg(bd.cu_q + b + 1) - __ldg(bd.cu_q + b);
-    const int n = __ldg(bd.seq_lens + b);
+    const int m = cuq[b + 1] - cuq[b];
+    const int n = sl[b];
     if (m < 0 || n < m || n > bd.max_seq_len || (n > 0 && (n + kPage - 1) / kPage > bd.max_pages) ||
         (m > 0 && n < 1))
       report_error(status, kDevErrIndex);
-    pv.req_goff[b] = m > 0 ? (m + qpg - 1) / qpg : 0;
+    goff[b] = m > 0 ? (m + qpg - 1) / qpg : 0;
   }
-  if (threadIdx.x == 0) pv.req_goff[B] = 0;
+  if (threadIdx.x == 0) goff[B] = 0;
   __syncthreads();
-  const int G = block_exclusive_scan(pv.req_goff, B + 1, warp_sums);
-  // req_goff[B] now holds the total; rows and groups next
+  const int G = block_exclusive_scan(goff, B + 1, warp_sums);
+  // goff[B] now holds the total; rows and groups next
+  if (staged)
+    for (int i = threadIdx.x; i <= B; i += kPlanThreads) pv.req_goff[i] = goff[i];
   for (int t = threadIdx.x; t < T; t += kPlanThreads) {
-    const int b = upper_index(bd.cu_q, B + 1, t);
+    const int b = upper_index(cuq, B + 1, t);
     if (b < 0 || b >= B) {
       report_error(status, kDevErrIndex);
       pv.row_req[t] = 0;
       pv.row_pos[t] = 0;
       continue;
     }
-    const int c0 = __ldg(bd.cu_q + b), m = __ldg(bd.cu_q + b + 1) - c0;
-    const int n = __ldg(bd.seq_lens + b);
+    const int c0 = cuq[b], m = cuq[b + 1] - c0;
+    const int n = sl[b];
     pv.row_req[t] = b;
     pv.row_pos[t] = n - m + (t - c0);
   }
   for (int g = threadIdx.x; g < G; g += kPlanThreads) {
-    const int b = upper_index(pv.req_goff, B, g);
-    const int li = g - pv.req_goff[b];
-    const int c0 = __ldg(bd.cu_q + b), m = __ldg(bd.cu_q + b + 1) - c0;
-    const int n = __ldg(bd.seq_lens + b);
+    const int b = upper_index(goff, B, g);
+    const int li = g - goff[b];
+    const int c0 = cuq[b], m = cuq[b + 1] - c0;
+    const int n = sl[b];
     const int nq = min(qpg, m - li * qpg);
     const int pos0 = n - m + li * qpg;
     const int p_last = pos0 + nq - 1;
@@ -129,7 +150,10 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(BatchDev bd, int nhI
 }  // namespace
 
 int launch_plan(const BatchDev& b, int nhI, void* plan, void* stream) {
-  plan_kernel<<<1, kPlanThreads, 0, static_cast<cudaStream_t>(stream)>>>(b, nhI, plan);
+  const int staged = b.B <= kPlanSmemMaxB ? 1 : 0;
+  const size_t smem = staged ? sizeof(int32_t) * (3 * static_cast<size_t>(b.B) + 2) : 0;
+  const cudaError_t e = launch_pdl(plan_kernel, dim3(1), dim3(kPlanThreads), smem, stream, b, nhI, plan, staged);
+  if (e != cudaSuccess) return static_cast<int>(e);
   return static_cast<int>(cudaGetLastError());
 }
 

@@ -180,12 +180,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int unit = blockIdx.x >> 1;
   const int t = unit / p.nsplit, split = unit % p.nsplit;
   const int H = p.H;
-  const int b = __ldg(p.row_req + t);
-  const int pos = __ldg(p.row_pos + t);
-  const int nvis = min(p.k, pos + 1);
-  const int e0 = split * p.chunk;
-  const int nkeys = max(0, min(nvis - e0, p.chunk));
-  const int ntiles = (nkeys + kTile - 1) / kTile;
 
   if (threadIdx.x == 0) {
     if (is_s) {
@@ -220,16 +214,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&bar[B_STATS], 128);
     }
     fence_barrier_init();
-    if (is_s && ntiles > 0) {  // Q: 9 boxes of 128 heads x 64 dims; dims 0..511 land in the cp.async ring
-      tma_prefetch_desc(&qmap);
-      mbar_arrive_expect_tx(&bar[B_QROPE], 9 * kBlk);
-      for (int blk = 0; blk < 8; ++blk) tma_load_2d(base + Smem::kKRing + blk * kBlk, &qmap, 64 * blk, t * H, &bar[B_QROPE]);
-      tma_load_2d(base + Smem::kQRope, &qmap, 512, t * H, &bar[B_QROPE]);
-    }
+    tma_prefetch_desc(&qmap);
   }
   if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
+  }
+  // everything above stays inside this CTA; from here on the kernel reads the plan and S_t
+  pdl_trigger();
+  pdl_wait();
+  const int b = __ldg(p.row_req + t);
+  const int pos = __ldg(p.row_pos + t);
+  const int nvis = min(p.k, pos + 1);
+  const int e0 = split * p.chunk;
+  const int nkeys = max(0, min(nvis - e0, p.chunk));
+  const int ntiles = (nkeys + kTile - 1) / kTile;
+  if (threadIdx.x == 0 && is_s && ntiles > 0) {  // Q: 9 boxes of 128 heads x 64 dims; dims 0..511 -> ring
+    mbar_arrive_expect_tx(&bar[B_QROPE], 9 * kBlk);
+    for (int blk = 0; blk < 8; ++blk) tma_load_2d(base + Smem::kKRing + blk * kBlk, &qmap, 64 * blk, t * H, &bar[B_QROPE]);
+    tma_load_2d(base + Smem::kQRope, &qmap, 512, t * H, &bar[B_QROPE]);
   }
 
   // physical rows of this cluster's entries (both CTAs); -1 marks an entry to skip
@@ -686,6 +689,8 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const float* __restric
                                                           float* __restrict__ lse) {
   const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  pdl_trigger();
+  pdl_wait();  // the partial results of the sparse MLA kernel
   if (gw >= T * H) return;
   const int t = gw / H, h = gw % H;
   float mx = -INFINITY;
@@ -789,15 +794,13 @@ int launch_sparse_mla(const BatchDev& b, const void* plan, const void* q, int H,
   cudaError_t ce =
       cudaFuncSetAttribute(sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem::kDynamic);
   if (ce != cudaSuccess) return static_cast<int>(ce);
-  dim3 grid(2 * b.T * prm.nsplit, 1, 1);
-  sparse_mla_kernel<<<grid, kThreads, Smem::kDynamic, static_cast<cudaStream_t>(stream)>>>(qmap, kvmap, omap, prm);
-  ce = cudaGetLastError();
+  ce = launch_pdl(sparse_mla_kernel, dim3(2 * b.T * prm.nsplit), dim3(kThreads), Smem::kDynamic, stream, qmap, kvmap,
+                  omap, prm);
   if (ce != cudaSuccess) return static_cast<int>(ce);
   if (prm.nsplit > 1) {
     const int warps = b.T * H;
-    mla_combine_kernel<<<(warps + 7) / 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        prm.part_o, prm.part_lse, b.T, H, prm.nsplit, prm.out, lse);
-    ce = cudaGetLastError();
+    ce = launch_pdl(mla_combine_kernel, dim3((warps + 7) / 8), dim3(256), 0, stream, prm.part_o, prm.part_lse, b.T, H,
+                    prm.nsplit, prm.out, lse);
   }
   return static_cast<int>(ce);
 }

@@ -94,6 +94,8 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
   __shared__ int2 cnt[kMaxChunks][kWarps];  // per (chunk, warp): (above theta, equal to theta)
 
   const int t = blockIdx.x;
+  pdl_trigger();
+  pdl_wait();  // scores and plan from the previous kernels
   const int L = __ldg(row_pos + t) + 1;
   const float* row = scores + static_cast<int64_t>(t) * ld;
   int32_t* out = S + static_cast<int64_t>(t) * k;
@@ -429,8 +431,8 @@ int launch_topk(const BatchDev& b, const void* plan, const float* scores, int64_
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(sizeof(uint32_t) * (kBins + kCandCap + kCacheCap)));
   if (e != cudaSuccess) return static_cast<int>(e);
-  topk_kernel<<<b.T, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(pv.row_pos, scores, ld, k, S, cap);
-  return static_cast<int>(cudaGetLastError());
+  return static_cast<int>(
+      launch_pdl(topk_kernel, dim3(b.T), dim3(kThreads), smem, stream, pv.row_pos, scores, ld, k, S, cap));
 }
 
 }  // namespace dsa
