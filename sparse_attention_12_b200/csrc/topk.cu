@@ -5,7 +5,7 @@
 //
 // One CTA of 1024 threads per query row; L = p + 1 visible scores.
 //  1. Scores become order-preserving uint32 keys (one float4 per thread per chunk of 4096
-//     positions, all loads in flight); the row's smallest and largest key bound the search.
+//     positions, four chunks in flight); the row's smallest and largest key bound the search.
 //  2. A 2048-bin histogram linear in the score value between the row's minimum and maximum
 //     (floating-point subtraction and scaling are monotonic, so bins stay ordered) locates the bin
 //     holding the k-th largest score; real score rows spread over many bins, so plain shared-memory
@@ -36,10 +36,12 @@ constexpr int kBins = 2048;
 constexpr int kChunk = 4 * kThreads;  // positions per chunk (one float4 per thread)
 constexpr int kCacheCap = 32768;      // keys kept in shared memory (128 KB)
 constexpr int kCandCap = 128;         // candidates resolved by counting
-constexpr int kGroup = 4;             // chunks whose loads are in flight together
+constexpr int kLoadGroup = 4;         // chunks whose global loads are in flight together
 constexpr int kMaxChunks = kMaxTopKRow / kChunk;  // 64 chunks: rows up to 262144 positions
-static_assert(kMaxChunks % kGroup == 0, "chunk groups");
+static_assert(kMaxChunks % kLoadGroup == 0, "chunk groups");
 static_assert(kCandCap <= kThreads, "one candidate per thread");
+constexpr int kBinsPerThread = kBins / kThreads;  // descending bins owned by one thread in the scan
+static_assert(kBins % kThreads == 0 && kWarps <= 32, "bin ownership");
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t b = __float_as_uint(f);
@@ -62,13 +64,13 @@ __device__ __forceinline__ int block_inclusive_scan(int v, int* scratch, int* to
   if (lane == 31) scratch[wid] = x;
   __syncthreads();
   if (wid == 0) {
-    int s = scratch[lane];
+    int s = lane < kWarps ? scratch[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, s, o);
       if (lane >= o) s += y;
     }
-    scratch[lane] = s;
+    if (lane < kWarps) scratch[lane] = s;
   }
   __syncthreads();
   const int r = x + (wid > 0 ? scratch[wid - 1] : 0);
@@ -81,6 +83,10 @@ struct Keys4 {
   uint32_t k[4];
 };
 
+// G: chunks processed per step after the first pass. Rows cached in shared memory take G = 1 (one
+// 16-byte shared load per chunk, no need to batch; a compact loop body keeps the instruction cache
+// warm), rows re-read from global memory take G = 4 (four loads in flight).
+template <int G>
 __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restrict__ row_pos,
                                                         const float* __restrict__ scores, int64_t ld, int k,
                                                         int32_t* __restrict__ S, int cache_cap) {
@@ -108,12 +114,12 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
   const bool cached = L <= cache_cap;
   const int nchunks = (L + kChunk - 1) / kChunk;
 
-  // keys of this thread in chunks cg .. cg + kGroup - 1 (all loads issued before any is used);
+  // keys of this thread in chunks cg .. cg + G - 1 (all loads issued before any is used);
   // positions >= L report nv = 0 and key 0
-  auto load_group = [&](int cg, Keys4 (&r)[kGroup], int (&nv)[kGroup]) {
-    float4 f[kGroup];
+  auto load_group = [&](int cg, Keys4 (&r)[G], int (&nv)[G]) {
+    float4 f[G];
 #pragma unroll
-    for (int g = 0; g < kGroup; ++g) {
+    for (int g = 0; g < G; ++g) {
       const int j0 = (cg + g) * kChunk + 4 * tid;
       nv[g] = max(0, min(4, L - j0));
       if (nv[g] > 0) {
@@ -126,7 +132,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
       }
     }
 #pragma unroll
-    for (int g = 0; g < kGroup; ++g) {
+    for (int g = 0; g < G; ++g) {
       if (nv[g] == 0) {
         r[g].k[0] = r[g].k[1] = r[g].k[2] = r[g].k[3] = 0u;
       } else if (!cached) {
@@ -138,17 +144,17 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
 
   // ---- 1. keys, row minimum and maximum ----
   uint32_t kmin = 0xffffffffu, kmax = 0u;
-  for (int cg = 0; cg < nchunks; cg += kGroup) {
-    float4 f[kGroup];
-    int nv[kGroup];
+  for (int cg = 0; cg < nchunks; cg += kLoadGroup) {
+    float4 f[kLoadGroup];
+    int nv[kLoadGroup];
 #pragma unroll
-    for (int g = 0; g < kGroup; ++g) {
+    for (int g = 0; g < kLoadGroup; ++g) {
       const int j0 = (cg + g) * kChunk + 4 * tid;
       nv[g] = max(0, min(4, L - j0));
       if (nv[g] > 0) f[g] = __ldg(reinterpret_cast<const float4*>(row + j0));
     }
 #pragma unroll
-    for (int g = 0; g < kGroup; ++g) {
+    for (int g = 0; g < kLoadGroup; ++g) {
       if (nv[g] == 0) continue;
       const uint32_t u[4] = {order_key(f[g].x), order_key(f[g].y), order_key(f[g].z), order_key(f[g].w)};
 #pragma unroll
@@ -163,8 +169,8 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
   if (lane == 0) red_min[wid] = kmin, red_max[wid] = kmax;
   for (int i = tid; i < kBins; i += kThreads) hist[i] = 0u;
   __syncthreads();
-  kmin = __reduce_min_sync(0xffffffffu, red_min[lane]);
-  kmax = __reduce_max_sync(0xffffffffu, red_max[lane]);
+  kmin = __reduce_min_sync(0xffffffffu, lane < kWarps ? red_min[lane] : 0xffffffffu);
+  kmax = __reduce_max_sync(0xffffffffu, lane < kWarps ? red_max[lane] : 0u);
 
   uint32_t lo = kmin, wmax = kmax - kmin;  // key-space range [lo, lo + wmax]
   uint32_t remaining = static_cast<uint32_t>(k);
@@ -185,19 +191,19 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
     best = __reduce_max_sync(0xffffffffu, have ? best : 0u);
     if (lane == 0) red_max[wid] = best;
     __syncthreads();
-    theta = __reduce_max_sync(0xffffffffu, red_max[lane]);
+    theta = __reduce_max_sync(0xffffffffu, lane < kWarps ? red_max[lane] : 0u);
     const uint32_t v = (static_cast<uint32_t>(tid) < ncand) ? cand[tid] : 0u;
     const int gt = __syncthreads_count(static_cast<uint32_t>(tid) < ncand && v > theta);
     remaining -= static_cast<uint32_t>(gt);
   };
   // copies the keys satisfying `pred` into cand (their number is known to be <= kCandCap)
   auto compact = [&](auto pred) {
-    for (int cg = 0; cg < nchunks; cg += kGroup) {
-      Keys4 r[kGroup];
-      int nv[kGroup];
+    for (int cg = 0; cg < nchunks; cg += G) {
+      Keys4 r[G];
+      int nv[G];
       load_group(cg, r, nv);
 #pragma unroll
-      for (int g = 0; g < kGroup; ++g) {
+      for (int g = 0; g < G; ++g) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const bool in = e < nv[g] && pred(r[g].k[e]);
@@ -215,12 +221,12 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
   };
   // hist[bin(key)] += 1 over the keys with bin(key) < kBins (one atomic per warp when all agree)
   auto histogram = [&](auto bin_of) {
-    for (int cg = 0; cg < nchunks; cg += kGroup) {
-      Keys4 r[kGroup];
-      int nv[kGroup];
+    for (int cg = 0; cg < nchunks; cg += G) {
+      Keys4 r[G];
+      int nv[G];
       load_group(cg, r, nv);
 #pragma unroll
-      for (int g = 0; g < kGroup; ++g) {
+      for (int g = 0; g < G; ++g) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const uint32_t bin = e < nv[g] ? bin_of(r[g].k[e]) : 0xffffffffu;
@@ -242,20 +248,25 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
   // the bin b (of nb, counted from the top) holding the remaining-th largest key:
   // sh_bin = b, sh_remaining = remaining - (keys in higher bins), sh_ncand = keys in b
   auto find_bin = [&](uint32_t nb) {
-    const int d0 = 2 * tid, d1 = d0 + 1;  // thread i owns descending bins 2i, 2i+1
-    const uint32_t c0 = (static_cast<uint32_t>(d0) < nb) ? hist[nb - 1 - d0] : 0u;
-    const uint32_t c1 = (static_cast<uint32_t>(d1) < nb) ? hist[nb - 1 - d1] : 0u;
+    // thread i owns descending bins kBinsPerThread*i .. +kBinsPerThread-1 (counted from the top)
+    uint32_t cnts[kBinsPerThread], sum = 0;
+#pragma unroll
+    for (int q = 0; q < kBinsPerThread; ++q) {
+      const uint32_t d = static_cast<uint32_t>(kBinsPerThread * tid + q);
+      cnts[q] = d < nb ? hist[nb - 1 - d] : 0u;
+      sum += cnts[q];
+    }
     int total;
-    const int incl = block_inclusive_scan(static_cast<int>(c0 + c1), scan_scratch, &total);
-    const uint32_t before = static_cast<uint32_t>(incl) - c0 - c1;
-    if (before < remaining && remaining <= before + c0) {
-      sh_lo = nb - 1 - d0;
-      sh_remaining = remaining - before;
-      sh_ncand = c0;
-    } else if (before + c0 < remaining && remaining <= before + c0 + c1) {
-      sh_lo = nb - 1 - d1;
-      sh_remaining = remaining - before - c0;
-      sh_ncand = c1;
+    const int incl = block_inclusive_scan(static_cast<int>(sum), scan_scratch, &total);
+    uint32_t before = static_cast<uint32_t>(incl) - sum;
+#pragma unroll
+    for (int q = 0; q < kBinsPerThread; ++q) {
+      if (before < remaining && remaining <= before + cnts[q]) {
+        sh_lo = nb - 1 - static_cast<uint32_t>(kBinsPerThread * tid + q);
+        sh_remaining = remaining - before;
+        sh_ncand = cnts[q];
+      }
+      before += cnts[q];
     }
     if (tid == 0) sh_done = 0u;
     __syncthreads();
@@ -282,12 +293,12 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
       } else {
         // the boundary bin is a contiguous key interval: narrow it in key space
         uint32_t bmin = 0xffffffffu, bmax = 0u;
-        for (int cg = 0; cg < nchunks; cg += kGroup) {
-          Keys4 r[kGroup];
-          int nv[kGroup];
+        for (int cg = 0; cg < nchunks; cg += G) {
+          Keys4 r[G];
+          int nv[G];
           load_group(cg, r, nv);
 #pragma unroll
-          for (int g = 0; g < kGroup; ++g)
+          for (int g = 0; g < G; ++g)
 #pragma unroll
             for (int e = 0; e < 4; ++e)
               if (e < nv[g] && vbin(r[g].k[e]) == bstar) bmin = min(bmin, r[g].k[e]), bmax = max(bmax, r[g].k[e]);
@@ -297,8 +308,8 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
         if (lane == 0) red_min[wid] = bmin, red_max[wid] = bmax;
         for (int i = tid; i < kBins; i += kThreads) hist[i] = 0u;
         __syncthreads();
-        lo = __reduce_min_sync(0xffffffffu, red_min[lane]);
-        wmax = __reduce_max_sync(0xffffffffu, red_max[lane]) - lo;
+        lo = __reduce_min_sync(0xffffffffu, lane < kWarps ? red_min[lane] : 0xffffffffu);
+        wmax = __reduce_max_sync(0xffffffffu, lane < kWarps ? red_max[lane] : 0u) - lo;
         kmax = lo + wmax;
         __syncthreads();  // red_min / red_max are reused below
         if (wmax == 0u) {
@@ -341,12 +352,12 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
   // theta: the k-th largest key; remaining: how many keys equal to theta are taken
 
   // ---- 4. ordered emission ----
-  for (int cg = 0; cg < nchunks; cg += kGroup) {
-    Keys4 r[kGroup];
-    int nv[kGroup];
+  for (int cg = 0; cg < nchunks; cg += G) {
+    Keys4 r[G];
+    int nv[G];
     load_group(cg, r, nv);
 #pragma unroll
-    for (int g = 0; g < kGroup; ++g) {
+    for (int g = 0; g < G; ++g) {
       int gt = 0, eq = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -362,26 +373,26 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
   if (wid == 0) {  // exclusive prefix over (chunk, warp) in position order
     int2 carry = make_int2(0, 0);
     for (int c = 0; c < nchunks; ++c) {
-      const int2 v = cnt[c][lane];
+      const int2 v = lane < kWarps ? cnt[c][lane] : make_int2(0, 0);
       int2 x = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int yx = __shfl_up_sync(0xffffffffu, x.x, o), yy = __shfl_up_sync(0xffffffffu, x.y, o);
         if (lane >= o) x.x += yx, x.y += yy;
       }
-      cnt[c][lane] = make_int2(carry.x + x.x - v.x, carry.y + x.y - v.y);
+      if (lane < kWarps) cnt[c][lane] = make_int2(carry.x + x.x - v.x, carry.y + x.y - v.y);
       carry.x += __shfl_sync(0xffffffffu, x.x, 31);
       carry.y += __shfl_sync(0xffffffffu, x.y, 31);
     }
   }
   __syncthreads();
   const int ties = static_cast<int>(remaining);
-  for (int cg = 0; cg < nchunks; cg += kGroup) {
-    Keys4 r[kGroup];
-    int nv[kGroup];
+  for (int cg = 0; cg < nchunks; cg += G) {
+    Keys4 r[G];
+    int nv[G];
     load_group(cg, r, nv);
 #pragma unroll
-    for (int g = 0; g < kGroup; ++g) {
+    for (int g = 0; g < G; ++g) {
       const int c = cg + g;
       int gt = 0, eq = 0;
 #pragma unroll
@@ -428,11 +439,12 @@ int launch_topk(const BatchDev& b, const void* plan, const float* scores, int64_
   PlanView pv = plan_view(const_cast<void*>(plan), b.B, b.T);
   const int cap = b.max_seq_len <= kCacheCap ? ((b.max_seq_len + 3) & ~3) : 0;
   const size_t smem = sizeof(uint32_t) * (kBins + kCandCap + static_cast<size_t>(cap));
-  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kern = (cap > 0) ? topk_kernel<1> : topk_kernel<4>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(sizeof(uint32_t) * (kBins + kCandCap + kCacheCap)));
   if (e != cudaSuccess) return static_cast<int>(e);
   return static_cast<int>(
-      launch_pdl(topk_kernel, dim3(b.T), dim3(kThreads), smem, stream, pv.row_pos, scores, ld, k, S, cap));
+      launch_pdl(kern, dim3(b.T), dim3(kThreads), smem, stream, pv.row_pos, scores, ld, k, S, cap));
 }
 
 }  // namespace dsa
