@@ -73,6 +73,26 @@ def bf16_decode(bits) -> np.ndarray:
     return b.view(np.float32).astype(np.float64)
 
 
+def e4m3_encode(values) -> np.ndarray:
+    """OCP FP8 E4M3 (e4m3fn) codes of finite float32 values: the nearest representable value,
+    ties to the even code, magnitudes above 448 saturating to 448; the sign of zero is kept.
+
+    Brute force over the magnitudes e4m3_decode gives codes 0x00..0x7E (0 .. 448), so the rounding
+    can be checked by eye: among the magnitudes nearest to |v|, the even code wins.
+    """
+    v = np.asarray(values, np.float32).astype(np.float64)  # exact widening
+    mags = e4m3_decode(np.arange(0x7F, dtype=np.uint8))     # 127 non-negative finite magnitudes
+    codes_all = np.arange(0x7F)
+    mag = np.minimum(np.abs(v), 448.0)
+    dist = np.abs(mag[..., None] - mags)
+    nearest = dist == dist.min(axis=-1, keepdims=True)     # one code, or two at an exact midpoint
+    big = 1 << 20
+    even = np.where(nearest & (codes_all % 2 == 0), codes_all, big).min(axis=-1)
+    anyc = np.where(nearest, codes_all, big).min(axis=-1)
+    code = np.where(even < big, even, anyc)
+    return (code | np.where(np.signbit(v), 0x80, 0)).astype(np.uint8)
+
+
 # ---------------------------------------------------------------------------------------------
 # batch geometry
 
@@ -186,6 +206,41 @@ def sparse_mla(seq_lens, cu_q, block_table, q, kv_cache, S, softmax_scale, rows=
     for t in (range(T) if rows is None else rows):
         out[t], lse[t] = sparse_mla_row(t, req, S[t], block_table, q, kv_cache, softmax_scale)
     return out, lse
+
+
+# ---------------------------------------------------------------------------------------------
+# writing new positions into the two caches: per token the latent row in bf16 and the indexer key
+# as FP8 plus a 4-byte scale, the indexer keys paged like the latent rows [P1-DSA]; one indexer key
+# per position, shared by every indexer head and kept in its own key cache [P5-LI]
+
+def indexer_key_quantize(k_row):
+    """(codes uint8[d], scale float32) of one new indexer key.
+
+    Reading of "FP8 + a 4-byte scale per token": s = max_d |k_d| / 448 in float32 (1 when the key is
+    all zeros), codes = e4m3(k_d / s) with the division in float32 (correctly rounded).
+    """
+    k = np.asarray(k_row, np.float32)
+    amax = np.float32(np.max(np.abs(k)))
+    s = np.float32(amax / np.float32(448.0)) if amax > 0 else np.float32(1.0)
+    return e4m3_encode((k / s).astype(np.float32)), s
+
+
+def cache_write(seq_lens, cu_q, block_table, k_new, c_new_bits, kI_cache, kI_scale, kv_cache):
+    """The three caches after writing every query row's own position (updated copies).
+
+    Query row t (request b, position p) stores its indexer key at kI_cache[page][p % 64] with the
+    scale at kI_scale[page][p % 64], and its latent row (bf16 bits) at kv_cache[page][p % 64],
+    page = block_table[b][p // 64]. Every other slot keeps its contents.
+    """
+    req, pos = query_positions(seq_lens, cu_q)
+    kI, ks, kv = np.array(kI_cache, copy=True), np.array(kI_scale, copy=True), np.array(kv_cache, copy=True)
+    for t in range(len(req)):
+        pages, slots = physical_rows(block_table[req[t]], [pos[t]])
+        codes, s = indexer_key_quantize(k_new[t])
+        kI[pages[0], slots[0]] = codes
+        ks[pages[0], slots[0]] = s
+        kv[pages[0], slots[0]] = c_new_bits[t]
+    return kI, ks, kv
 
 
 # ---------------------------------------------------------------------------------------------

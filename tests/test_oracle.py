@@ -35,6 +35,90 @@ def test_e4m3_decode_matches_torch_all_codes():
     assert O.e4m3_decode(np.uint8(0xB8)) == -1.0
 
 
+# ---------------------------------------------------------------------------------------------
+# e4m3 encoder: round to nearest, ties to even, saturation at 448 (OCP E4M3)
+
+def _finite_codes():
+    return np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+
+
+def test_e4m3_encode_round_trips_every_finite_code():
+    codes = _finite_codes()
+    vals = O.e4m3_decode(codes).astype(np.float32)
+    vals[codes == 0x80] = np.float32(-0.0)  # the decoder folds -0 to 0.0 * -1 = -0.0 already
+    assert np.array_equal(O.e4m3_encode(vals), codes)
+
+
+def test_e4m3_encode_midpoints_go_to_the_even_code():
+    mags = O.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+    for c in range(0x7E):
+        lo, hi = mags[c], mags[c + 1]
+        mid = np.float32((lo + hi) / 2)           # at most 5 significant bits: exact in float32
+        assert float(mid) == (lo + hi) / 2
+        want = c if c % 2 == 0 else c + 1
+        assert O.e4m3_encode([mid])[0] == want, (c, mid)
+        assert O.e4m3_encode([-mid])[0] == want | 0x80
+        below = np.nextafter(mid, np.float32(0.0), dtype=np.float32)
+        above = np.nextafter(mid, np.float32(1e9), dtype=np.float32)
+        assert O.e4m3_encode([below])[0] == c and O.e4m3_encode([above])[0] == c + 1
+
+
+def test_e4m3_encode_saturates_and_keeps_zero_sign():
+    enc = O.e4m3_encode(np.array([448.0, 464.0, 479.0, 1e30, -448.0, -1e30, 0.0, -0.0, 2.0 ** -12, -(2.0 ** -12)],
+                                 np.float32))
+    assert list(enc) == [0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0xFE, 0x00, 0x80, 0x00, 0x80]
+
+
+def test_indexer_key_quantize_scale_and_error_bound():
+    rng = np.random.default_rng(3)
+    for k in [rng.standard_normal(128) * 3.0, rng.standard_normal(128) * 1e-3, np.zeros(128)]:
+        k = k.astype(np.float32)
+        codes, s = O.indexer_key_quantize(k)
+        amax = np.float32(np.abs(k).max())
+        assert s == (np.float32(amax / np.float32(448.0)) if amax > 0 else np.float32(1.0))
+        back = O.e4m3_decode(codes) * float(s)
+        if amax > 0:
+            assert (codes & 0x7F).max() == 0x7E   # the largest element maps to +-448
+            # E4M3 keeps 3 mantissa bits: relative error <= 2^-4 above the subnormal range
+            normal = np.abs(k) / float(s) >= 2.0 ** -6
+            assert np.all(np.abs(back - k)[normal] <= 2.0 ** -4 * np.abs(k)[normal] * (1 + 1e-6))
+        else:
+            assert np.all(codes == 0)
+
+
+def test_indexer_key_quantize_agrees_with_the_synthetic_generator():
+    # cross-check (not a pin): synth quantises with torch's float8 cast under the same reading
+    rng = np.random.default_rng(4)
+    x = (rng.standard_normal((16, 128)) * np.exp(rng.uniform(-4, 4, (16, 1)))).astype(np.float32)
+    codes, scale = synth.quantize_e4m3_per_token(x)
+    for t in range(16):
+        c, s = O.indexer_key_quantize(x[t])
+        assert s == scale[t] and np.array_equal(c, codes[t])
+
+
+def test_cache_write_places_rows_and_leaves_the_rest():
+    rng = np.random.default_rng(5)
+    P = 6
+    kI = rng.integers(0, 256, (P, 64, 128)).astype(np.uint8)
+    ks = rng.standard_normal((P, 64)).astype(np.float32)
+    kv = rng.integers(0, 1 << 16, (P, 64, 576)).astype(np.uint16)
+    seq_lens, cu_q = np.array([130, 64]), np.array([0, 2, 3])     # rows at positions 128, 129 and 63
+    block_table = np.array([[4, 0, 2], [5, -1, -1]])
+    k_new = rng.standard_normal((3, 128)).astype(np.float32)
+    c_new = rng.integers(0, 1 << 16, (3, 576)).astype(np.uint16)
+    kI2, ks2, kv2 = O.cache_write(seq_lens, cu_q, block_table, k_new, c_new, kI, ks, kv)
+    where = [(2, 0), (2, 1), (5, 63)]                               # (page, slot) of each row
+    for t, (pg, sl) in enumerate(where):
+        codes, s = O.indexer_key_quantize(k_new[t])
+        assert np.array_equal(kI2[pg, sl], codes) and ks2[pg, sl] == s
+        assert np.array_equal(kv2[pg, sl], c_new[t])
+    mask = np.ones((P, 64), bool)
+    for pg, sl in where:
+        mask[pg, sl] = False
+    assert np.array_equal(kI2[mask], kI[mask]) and np.array_equal(ks2[mask], ks[mask])
+    assert np.array_equal(kv2[mask], kv[mask])
+
+
 def test_bf16_decode_matches_torch():
     rng = np.random.default_rng(1)
     bits = rng.integers(0, 1 << 16, size=4096, dtype=np.uint16)
