@@ -86,6 +86,23 @@ dsa_status_t dsa_plan(const dsa_batch_t* batch, int nhI, void* plan, size_t plan
  * `plan` recorded (DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE_INDEX) and clears it. */
 dsa_status_t dsa_status_read(void* plan, void* stream);
 
+/* ---- writing new positions into the caches (the step before step 1) ----------------------
+ * Every query row t (request b, position p) is a new token; its indexer key and its latent row are
+ * stored at slot p % 64 of page block_table[b][p / 64] of the two caches:
+ *   kI_scale[page][slot]    = s = max_d |k_new[t][d]| / 448 (fp32; 1 when the key is all zeros)
+ *   kI_cache[page][slot][d] = e4m3(k_new[t][d] / s)   division in fp32; OCP E4M3, nearest with
+ *                                                      ties to even, saturating at +-448
+ *   kv_cache[page][slot][:] = c_new[t][:]            576 bf16, copied
+ * ("MTP 与稀疏注意力：NSA 与 DSA", section "稀疏注意力：NSA 与 DSA": per token the latent vector and the
+ * indexer key as FP8 + a 4-byte scale, both paged; "DeepSeek Sparse Attention：从 SWA 到稀疏
+ * Attention 计算", Lightning Indexer section: one shared indexer key per position in its own key
+ * cache.) The plan must be made for this batch (dsa_plan).
+ * k_new f32 [T, 128] (finite), c_new bf16 [T, 576]; caches as for dsa_index_scores / dsa_sparse_mla.
+ * A page id outside [0, num_pages) is recorded as DSA_ERR_DEVICE_INDEX (dsa_status_read) and its
+ * row is skipped. */
+dsa_status_t dsa_cache_write(const dsa_batch_t* batch, const void* plan, const float* k_new, const void* c_new,
+                             uint8_t* kI_cache, float* kI_scale, void* kv_cache, void* stream);
+
 /* ---- step 1: indexer scores -------------------------------------------------------------
  * qI       e4m3 [T, nhI, 128]   indexer queries (FP8 codes)
  * qI_scale f32  [T]             s^q_t

@@ -38,7 +38,7 @@ class DsaBatchC(ctypes.Structure):
 
 EXPORTS = ("dsa_abi_version", "dsa_status_string", "dsa_plan_workspace_size", "dsa_plan", "dsa_status_read",
            "dsa_index_scores", "dsa_topk", "dsa_sparse_mla_workspace_size", "dsa_sparse_mla",
-           "dsa_layer_workspace_size", "dsa_layer", "dsa_layer_noalloc")
+           "dsa_layer_workspace_size", "dsa_layer", "dsa_layer_noalloc", "dsa_cache_write")
 
 _lib = None
 
@@ -66,6 +66,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "dsa_layer_workspace_size": (SZ, [BP, I, I, I]),
         "dsa_layer": (I, [BP, P, P, P, I, P, P, P, I, P, I, ctypes.c_float, P, P, P, P, SZ, P]),
         "dsa_layer_noalloc": (I, [BP, P, P, P, I, P, P, P, I, P, I, ctypes.c_float, P, P, P, P]),
+        "dsa_cache_write": (I, [BP, P, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -148,6 +149,20 @@ def plan(batch: Batch, nhI: int, plan_ws: Optional[torch.Tensor] = None) -> torc
 def status_read(plan_ws: torch.Tensor) -> int:
     """Synchronise the current stream and return (and clear) the kernels' status word."""
     return load().dsa_status_read(plan_ws.data_ptr(), _stream())
+
+
+def cache_write(batch: Batch, plan_ws, k_new, c_new, kI_cache, kI_scale, kv_cache) -> None:
+    """Store every query row's new indexer key (fp32 [T, 128], quantised to FP8 + scale) and latent
+    row (bf16 [T, 576]) at its own position of the paged caches (dsa_cache_write)."""
+    T = batch.total_q
+    _need(k_new, "k_new", torch.float32, (T, D_INDEX))
+    _need(c_new, "c_new", torch.bfloat16, (T, D_LATENT))
+    _need(kI_cache, "kI_cache", torch.float8_e4m3fn)
+    _need(kI_scale, "kI_scale", torch.float32)
+    _need(kv_cache, "kv_cache", torch.bfloat16)
+    _check(load().dsa_cache_write(batch.ref(), plan_ws.data_ptr(), k_new.data_ptr(), c_new.data_ptr(),
+                                  kI_cache.data_ptr(), kI_scale.data_ptr(), kv_cache.data_ptr(), _stream()),
+           "dsa_cache_write")
 
 
 def index_scores(batch: Batch, plan_ws, qI, qI_scale, wI, kI_cache, kI_scale, scores=None, ld=None) -> torch.Tensor:

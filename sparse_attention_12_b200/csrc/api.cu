@@ -146,6 +146,18 @@ dsa_status_t dsa_sparse_mla(const dsa_batch_t* batch, const void* plan, const vo
   return from_cuda(launch_sparse_mla(to_dev(batch), plan, q, H, kv_cache, S, k, softmax_scale, out, lse, ws, stream));
 }
 
+dsa_status_t dsa_cache_write(const dsa_batch_t* batch, const void* plan, const float* k_new, const void* c_new,
+                             uint8_t* kI_cache, float* kI_scale, void* kv_cache, void* stream) {
+  dsa_status_t st = check_batch(batch);
+  if (st != DSA_OK) return st;
+  if (batch->total_q == 0) return DSA_OK;
+  if (!plan || !k_new || !c_new || !kI_cache || !kI_scale || !kv_cache) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(plan) || !aligned16(k_new) || !aligned16(c_new) || !aligned16(kI_cache) || !aligned16(kI_scale) ||
+      !aligned16(kv_cache))
+    return DSA_ERR_INVALID_ARG;
+  return from_cuda(launch_cache_write(to_dev(batch), plan, k_new, c_new, kI_cache, kI_scale, kv_cache, stream));
+}
+
 size_t dsa_layer_workspace_size(const dsa_batch_t* batch, int nhI, int H, int k) {
   if (check_batch(batch) != DSA_OK || !valid_nhI(nhI) || H < 1 || H > 128 || k < 1 || k > kMaxTopK) return 0;
   const size_t T = static_cast<size_t>(batch->total_q);

@@ -102,6 +102,8 @@ struct BatchDev {
 };
 
 int launch_plan(const BatchDev& b, int nhI, void* plan, void* stream);
+int launch_cache_write(const BatchDev& b, const void* plan, const float* k_new, const void* c_new, uint8_t* kI_cache,
+                       float* kI_scale, void* kv_cache, void* stream);
 int launch_index_scores(const BatchDev& b, const void* plan, const uint8_t* qI, const float* qI_scale,
                         const float* wI, int nhI, const uint8_t* kI_cache, const float* kI_scale, float* scores,
                         int64_t ld, void* stream);

@@ -88,6 +88,18 @@ def test_index_scores_validation(lib):
     assert call(scores=None) == 1
 
 
+def test_cache_write_validation(lib):
+    b = batch()
+    call = lambda **kw: lib.dsa_cache_write(ctypes.byref(b), kw.get("plan", FAKE), kw.get("k", FAKE), kw.get("c", FAKE),
+                                            kw.get("kI", FAKE), kw.get("ks", FAKE), kw.get("kv", FAKE), None)
+    assert call(k=None) == 1
+    assert call(kv=None) == 1
+    assert call(c=FAKE + 8) == 1        # misaligned
+    assert call(plan=FAKE + 4) == 1
+    empty = dsa.DsaBatchC(0, 0, 0, 0, 0, 0, None, None, None)
+    assert lib.dsa_cache_write(ctypes.byref(empty), None, None, None, None, None, None, None) == 0
+
+
 def test_topk_and_mla_validation(lib):
     b = batch()
     assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE, 384, 0, FAKE, None) == 2
