@@ -296,10 +296,12 @@ def main():
     S = torch.empty((T, db.k), dtype=torch.int32, device=dev)
     mla_ws_n = dsa.load().dsa_sparse_mla_workspace_size(db.batch.ref(), db.H, db.k)
     mla_ws = torch.empty(max(16, mla_ws_n), dtype=torch.uint8, device=dev)
+    topk_ws_n = dsa.load().dsa_topk_workspace_size(db.batch.ref(), db.k)
+    topk_ws = torch.empty(max(16, topk_ws_n), dtype=torch.uint8, device=dev) if topk_ws_n else None
     stages = {
         "index_scores": lambda: dsa.index_scores(db.batch, plan_t, db.qI, db.qI_scale, db.wI, db.kI_cache,
                                                  db.kI_scale, scores=scores, ld=ld),
-        "topk": lambda: dsa.topk(db.batch, plan_t, scores, db.k, S=S),
+        "topk": lambda: dsa.topk(db.batch, plan_t, scores, db.k, S=S, ws=topk_ws),
         "sparse_mla": lambda: dsa.sparse_mla(db.batch, plan_t, db.q, db.kv_cache, S, db.softmax_scale, out=out,
                                              ws=mla_ws),
     }
@@ -441,7 +443,7 @@ def main():
                "sample": f"{rows} of the {T} query rows of {wl.name} through the whole path in "
                          f"{dt:.1f} s (float64 numpy, BLAS threads)"}
 
-    launches_per_step = 3 + (1 if mla_ws_n > 0 else 0)
+    launches_per_step = 3 + (1 if mla_ws_n > 0 else 0) + (1 if topk_ws_n > 0 else 0)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "layer_us": 1e3 * ms,

@@ -46,7 +46,7 @@
 extern "C" {
 #endif
 
-#define DSA_ABI_VERSION 1
+#define DSA_ABI_VERSION 2
 #define DSA_PAGE_SIZE 64   /* positions per cache page */
 #define DSA_D_INDEX 128    /* indexer head width d_h^I */
 #define DSA_D_LATENT 576   /* latent width: 512 + 64 rope */
@@ -121,9 +121,12 @@ dsa_status_t dsa_index_scores(const dsa_batch_t* batch, const void* plan, const 
  *        ld >= max_seq_len. max_seq_len <= 262144 (else DSA_ERR_UNSUPPORTED).
  * S      int32 [T, k] out: the min(k, p+1) positions with the largest scores, followed by -1.
  *        Among equal scores the smaller position wins. Selected positions are listed in
- *        increasing position order. 1 <= k <= 4096. */
+ *        increasing position order. 1 <= k <= 4096.
+ * ws/ws_bytes: dsa_topk_workspace_size bytes (0 when max_seq_len <= 32768): rows longer than 32768
+ *        positions select per slice of 32768 first, then among the slices' winners. */
+size_t dsa_topk_workspace_size(const dsa_batch_t* batch, int k);
 dsa_status_t dsa_topk(const dsa_batch_t* batch, const void* plan, const float* scores, int64_t ld, int k,
-                      int32_t* S, void* stream);
+                      int32_t* S, void* ws, size_t ws_bytes, void* stream);
 
 /* ---- step 3: sparse MLA -----------------------------------------------------------------
  * q        bf16 [T, H, 576]     absorbed MLA queries, 1 <= H <= 128

@@ -37,7 +37,7 @@ class DsaBatchC(ctypes.Structure):
 
 
 EXPORTS = ("dsa_abi_version", "dsa_status_string", "dsa_plan_workspace_size", "dsa_plan", "dsa_status_read",
-           "dsa_index_scores", "dsa_topk", "dsa_sparse_mla_workspace_size", "dsa_sparse_mla",
+           "dsa_index_scores", "dsa_topk_workspace_size", "dsa_topk", "dsa_sparse_mla_workspace_size", "dsa_sparse_mla",
            "dsa_layer_workspace_size", "dsa_layer", "dsa_layer_noalloc", "dsa_cache_write")
 
 _lib = None
@@ -60,7 +60,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "dsa_plan": (I, [BP, I, P, SZ, P]),
         "dsa_status_read": (I, [P, P]),
         "dsa_index_scores": (I, [BP, P, P, P, P, I, P, P, P, I64, P]),
-        "dsa_topk": (I, [BP, P, P, I64, I, P, P]),
+        "dsa_topk_workspace_size": (SZ, [BP, I]),
+        "dsa_topk": (I, [BP, P, P, I64, I, P, P, SZ, P]),
         "dsa_sparse_mla_workspace_size": (SZ, [BP, I, I]),
         "dsa_sparse_mla": (I, [BP, P, P, I, P, P, I, ctypes.c_float, P, P, P, SZ, P]),
         "dsa_layer_workspace_size": (SZ, [BP, I, I, I]),
@@ -184,14 +185,18 @@ def index_scores(batch: Batch, plan_ws, qI, qI_scale, wI, kI_cache, kI_scale, sc
     return scores
 
 
-def topk(batch: Batch, plan_ws, scores: torch.Tensor, k: int, S=None) -> torch.Tensor:
+def topk(batch: Batch, plan_ws, scores: torch.Tensor, k: int, S=None, ws=None) -> torch.Tensor:
     T = batch.total_q
     _need(scores, "scores", torch.float32)
     if S is None:
         S = torch.empty((T, k), dtype=torch.int32, device="cuda")
     _need(S, "S", torch.int32, (T, k))
-    _check(load().dsa_topk(batch.ref(), plan_ws.data_ptr(), scores.data_ptr(), int(scores.shape[1]), k,
-                           S.data_ptr(), _stream()), "dsa_topk")
+    lib = load()
+    need = lib.dsa_topk_workspace_size(batch.ref(), k)
+    if ws is None and need > 0:
+        ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    _check(lib.dsa_topk(batch.ref(), plan_ws.data_ptr(), scores.data_ptr(), int(scores.shape[1]), k, S.data_ptr(),
+                        _ptr(ws), 0 if ws is None else ws.numel(), _stream()), "dsa_topk")
     return S
 
 

@@ -3,6 +3,7 @@
 // dsa_status_read, whose job is to read the device status word back.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 
@@ -113,8 +114,13 @@ dsa_status_t dsa_index_scores(const dsa_batch_t* batch, const void* plan, const 
                                        stream));
 }
 
+size_t dsa_topk_workspace_size(const dsa_batch_t* batch, int k) {
+  if (check_batch(batch) != DSA_OK || k < 1 || k > kMaxTopK || batch->max_seq_len > kMaxTopKRow) return 0;
+  return topk_ws_bytes(batch->total_q, batch->max_seq_len, k);
+}
+
 dsa_status_t dsa_topk(const dsa_batch_t* batch, const void* plan, const float* scores, int64_t ld, int k,
-                      int32_t* S, void* stream) {
+                      int32_t* S, void* ws, size_t ws_bytes, void* stream) {
   dsa_status_t st = check_batch(batch);
   if (st != DSA_OK) return st;
   if (k < 1 || k > kMaxTopK) return DSA_ERR_UNSUPPORTED;
@@ -122,7 +128,10 @@ dsa_status_t dsa_topk(const dsa_batch_t* batch, const void* plan, const float* s
   if (batch->max_seq_len > kMaxTopKRow) return DSA_ERR_UNSUPPORTED;
   if (!plan || !scores || !S || !aligned16(plan) || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
   if (ld < batch->max_seq_len || ld % 4 != 0) return DSA_ERR_INVALID_ARG;
-  return from_cuda(launch_topk(to_dev(batch), plan, scores, ld, k, S, stream));
+  const size_t need = topk_ws_bytes(batch->total_q, batch->max_seq_len, k);
+  if (need > 0 && (!ws || !aligned16(ws))) return DSA_ERR_INVALID_ARG;
+  if (ws_bytes < need) return DSA_ERR_WORKSPACE;
+  return from_cuda(launch_topk(to_dev(batch), plan, scores, ld, k, S, ws, stream));
 }
 
 size_t dsa_sparse_mla_workspace_size(const dsa_batch_t* batch, int H, int k) {
@@ -164,7 +173,9 @@ size_t dsa_layer_workspace_size(const dsa_batch_t* batch, int nhI, int H, int k)
   size_t s = align256(plan_bytes(batch->num_requests, batch->total_q));
   s += align256(sizeof(float) * T * scores_ld(batch));
   s += align256(sizeof(int32_t) * T * static_cast<size_t>(k));
-  s += align256(sparse_mla_ws_bytes(batch->total_q, H, k));
+  // one scratch region: the top-k candidates, then (after top-k is done) the split partials
+  s += align256(std::max(sparse_mla_ws_bytes(batch->total_q, H, k),
+                         topk_ws_bytes(batch->total_q, batch->max_seq_len, k)));
   return s;
 }
 
@@ -194,13 +205,13 @@ dsa_status_t dsa_layer(const dsa_batch_t* batch, const uint8_t* qI, const float*
   p += align256(sizeof(float) * T * static_cast<size_t>(ld));
   int32_t* S = reinterpret_cast<int32_t*>(p);
   p += align256(sizeof(int32_t) * T * static_cast<size_t>(k));
-  void* mla_ws = p;
+  void* mla_ws = p;  // also the top-k candidate space (the two are never live together)
   if (S_out) S = S_out;
 
   const BatchDev bd = to_dev(batch);
   int e = launch_plan(bd, nhI, plan, stream);
   if (!e) e = launch_index_scores(bd, plan, qI, qI_scale, wI, nhI, kI_cache, kI_scale, scores, ld, stream);
-  if (!e) e = launch_topk(bd, plan, scores, ld, k, S, stream);
+  if (!e) e = launch_topk(bd, plan, scores, ld, k, S, mla_ws, stream);
   if (!e) e = launch_sparse_mla(bd, plan, q, H, kv_cache, S, k, softmax_scale, out, lse, mla_ws, stream);
   return from_cuda(e);
 }

@@ -18,10 +18,14 @@
 //  4. Emission in increasing position order: every key above theta, then the first
 //     `ties` keys equal to theta (equal scores: the smaller position wins), so the result is
 //     deterministic. Per-(chunk, warp) counts and one warp-level scan give each warp its offsets.
-// Rows of up to kCacheCap keys keep their keys in shared memory; longer rows re-read the scores
-// (L2-resident: the indexer just wrote them) in each pass.
+// Keys always sit in shared memory (at most kSlice = 32768 of them per CTA). A row longer than
+// kSlice is split into slices of kSlice positions, one CTA each, each selecting its own top k; a
+// merge CTA per row then selects among the slices' winners (at most 8k candidates, their scores
+// gathered from the row). This is exact: an element of the row's top k has fewer than k elements
+// above it in its own slice too (same order: score, then position).
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 
 #include "dsa_internal.h"
@@ -34,11 +38,12 @@ constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
 constexpr int kChunk = 4 * kThreads;  // positions per chunk (one float4 per thread)
-constexpr int kCacheCap = 32768;      // keys kept in shared memory (128 KB)
+constexpr int kSlice = 32768;         // positions per CTA: their keys sit in shared memory (128 KB)
 constexpr int kCandCap = 128;         // candidates resolved by counting
 constexpr int kLoadGroup = 4;         // chunks whose global loads are in flight together
-constexpr int kMaxChunks = kMaxTopKRow / kChunk;  // 64 chunks: rows up to 262144 positions
-static_assert(kMaxChunks % kLoadGroup == 0, "chunk groups");
+constexpr int kMaxChunks = kSlice / kChunk;  // 8 chunks of 4096 positions per CTA
+constexpr int kMaxSlices = kMaxTopKRow / kSlice;  // rows up to 262144 positions: 8 slices
+static_assert(kMaxChunks % kLoadGroup == 0 && kMaxSlices * kMaxTopK <= kSlice, "a merge fits one CTA");
 static_assert(kCandCap <= kThreads, "one candidate per thread");
 constexpr int kBinsPerThread = kBins / kThreads;  // descending bins owned by one thread in the scan
 static_assert(kBins % kThreads == 0 && kWarps <= 32, "bin ownership");
@@ -83,61 +88,60 @@ struct Keys4 {
   uint32_t k[4];
 };
 
-// G: chunks processed per step after the first pass. Rows cached in shared memory take G = 1 (one
-// 16-byte shared load per chunk, no need to batch; a compact loop body keeps the instruction cache
-// warm), rows re-read from global memory take G = 4 (four loads in flight).
-template <int G>
+// kMerge = false (slice mode): CTA (t, s) of a T x nsl_max grid selects among positions
+//   [s*kSlice, min(L, (s+1)*kSlice)) of row t. A row of one slice writes S_t itself; otherwise the
+//   slice's k winners (increasing positions, -1 padded) go to block (t, s) of the candidate space.
+// kMerge = true: CTA t selects among the candidates of row t (their scores gathered from the row),
+//   in candidate order = increasing position; rows of one slice have nothing to do here.
+template <bool kMerge>
 __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restrict__ row_pos,
                                                         const float* __restrict__ scores, int64_t ld, int k,
-                                                        int32_t* __restrict__ S, int cache_cap) {
+                                                        int32_t* __restrict__ S, int32_t* __restrict__ cand_ws,
+                                                        int nsl_max, int kpad) {
   extern __shared__ __align__(16) uint32_t tk_smem[];
   uint32_t* hist = tk_smem;                 // [kBins]
   uint32_t* cand = tk_smem + kBins;         // [kCandCap]
-  uint32_t* cache = cand + kCandCap;        // [cache_cap]
+  uint32_t* cache = cand + kCandCap;        // [kSlice] keys of this CTA's positions
   __shared__ int scan_scratch[kWarps];
   __shared__ uint32_t red_min[kWarps], red_max[kWarps];
   __shared__ uint32_t sh_lo, sh_remaining, sh_ncand, sh_done;
   __shared__ int2 cnt[kMaxChunks][kWarps];  // per (chunk, warp): (above theta, equal to theta)
 
-  const int t = blockIdx.x;
+  const int t = kMerge ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x) / nsl_max;
+  const int sl = kMerge ? 0 : static_cast<int>(blockIdx.x) % nsl_max;
   pdl_trigger();
-  pdl_wait();  // scores and plan from the previous kernels
+  pdl_wait();  // scores, plan and candidates from the previous kernels
   const int L = __ldg(row_pos + t) + 1;
+  const int nsl = (L + kSlice - 1) / kSlice;
+  if (kMerge ? nsl <= 1 : sl >= nsl) return;
   const float* row = scores + static_cast<int64_t>(t) * ld;
-  int32_t* out = S + static_cast<int64_t>(t) * k;
+  const int base = sl * kSlice;
+  // the n elements this CTA selects from: positions base + i, or the candidates of row t
+  const int n = kMerge ? (nsl - 1) * k + min(k, L - (nsl - 1) * kSlice) : min(kSlice, L - base);
+  const int32_t* cands = cand_ws + static_cast<int64_t>(t) * nsl_max * kpad;
+  auto position = [&](int i) -> int { return kMerge ? __ldg(cands + (i / k) * kpad + i % k) : base + i; };
+  int32_t* out = (kMerge || nsl == 1) ? S + static_cast<int64_t>(t) * k
+                                      : cand_ws + (static_cast<int64_t>(t) * nsl_max + sl) * kpad;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
 
-  if (L <= k) {
-    for (int j = tid; j < k; j += kThreads) out[j] = (j < L) ? j : -1;
+  if (n <= k) {
+    for (int j = tid; j < k; j += kThreads) out[j] = (j < n) ? position(j) : -1;
     return;
   }
-  const bool cached = L <= cache_cap;
-  const int nchunks = (L + kChunk - 1) / kChunk;
+  const int nchunks = (n + kChunk - 1) / kChunk;
 
-  // keys of this thread in chunks cg .. cg + G - 1 (all loads issued before any is used);
-  // positions >= L report nv = 0 and key 0
+  // keys of this thread in chunks cg .. cg + G - 1 from shared memory; elements >= n report nv = 0
+  constexpr int G = 1;
   auto load_group = [&](int cg, Keys4 (&r)[G], int (&nv)[G]) {
-    float4 f[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       const int j0 = (cg + g) * kChunk + 4 * tid;
-      nv[g] = max(0, min(4, L - j0));
+      nv[g] = max(0, min(4, n - j0));
       if (nv[g] > 0) {
-        if (cached) {
-          const uint4 v = *reinterpret_cast<const uint4*>(cache + j0);
-          r[g].k[0] = v.x, r[g].k[1] = v.y, r[g].k[2] = v.z, r[g].k[3] = v.w;
-        } else {
-          f[g] = __ldg(reinterpret_cast<const float4*>(row + j0));  // j0 + 3 < ld: ld % 4 == 0
-        }
-      }
-    }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      if (nv[g] == 0) {
+        const uint4 v = *reinterpret_cast<const uint4*>(cache + j0);
+        r[g].k[0] = v.x, r[g].k[1] = v.y, r[g].k[2] = v.z, r[g].k[3] = v.w;
+      } else {
         r[g].k[0] = r[g].k[1] = r[g].k[2] = r[g].k[3] = 0u;
-      } else if (!cached) {
-        r[g].k[0] = order_key(f[g].x), r[g].k[1] = order_key(f[g].y);
-        r[g].k[2] = order_key(f[g].z), r[g].k[3] = order_key(f[g].w);
       }
     }
   };
@@ -150,8 +154,17 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
 #pragma unroll
     for (int g = 0; g < kLoadGroup; ++g) {
       const int j0 = (cg + g) * kChunk + 4 * tid;
-      nv[g] = max(0, min(4, L - j0));
-      if (nv[g] > 0) f[g] = __ldg(reinterpret_cast<const float4*>(row + j0));
+      nv[g] = max(0, min(4, n - j0));
+      if (nv[g] > 0) {
+        if (kMerge) {  // gather the candidates' scores
+          f[g].x = __ldg(row + position(j0));
+          f[g].y = nv[g] > 1 ? __ldg(row + position(j0 + 1)) : 0.f;
+          f[g].z = nv[g] > 2 ? __ldg(row + position(j0 + 2)) : 0.f;
+          f[g].w = nv[g] > 3 ? __ldg(row + position(j0 + 3)) : 0.f;
+        } else {  // base + j0 + 3 < ld: base and j0 are multiples of 4, ld % 4 == 0, base + j0 < L <= ld
+          f[g] = __ldg(reinterpret_cast<const float4*>(row + base + j0));
+        }
+      }
     }
 #pragma unroll
     for (int g = 0; g < kLoadGroup; ++g) {
@@ -160,8 +173,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
 #pragma unroll
       for (int e = 0; e < 4; ++e)
         if (e < nv[g]) kmin = min(kmin, u[e]), kmax = max(kmax, u[e]);
-      if (cached)
-        *reinterpret_cast<uint4*>(cache + (cg + g) * kChunk + 4 * tid) = make_uint4(u[0], u[1], u[2], u[3]);
+      *reinterpret_cast<uint4*>(cache + (cg + g) * kChunk + 4 * tid) = make_uint4(u[0], u[1], u[2], u[3]);
     }
   }
   kmin = __reduce_min_sync(0xffffffffu, kmin);
@@ -419,10 +431,10 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
         if (e >= nv[g]) break;
         const uint32_t u = r[g].k[e];
         if (u > theta) {
-          out[gt_before + min(eq_before, ties)] = j0 + e;
+          out[gt_before + min(eq_before, ties)] = position(j0 + e);
           ++gt_before;
         } else if (u == theta) {
-          if (eq_before < ties) out[gt_before + eq_before] = j0 + e;
+          if (eq_before < ties) out[gt_before + eq_before] = position(j0 + e);
           ++eq_before;
         }
       }
@@ -432,19 +444,36 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
 
 }  // namespace
 
-int launch_topk(const BatchDev& b, const void* plan, const float* scores, int64_t ld, int k, int32_t* S,
+size_t topk_ws_bytes(int T, int max_seq_len, int k) {
+  const int nsl = (max_seq_len + kSlice - 1) / kSlice;
+  if (nsl <= 1) return 0;
+  return sizeof(int32_t) * static_cast<size_t>(T) * static_cast<size_t>(nsl) * static_cast<size_t>((k + 3) & ~3);
+}
+
+int launch_topk(const BatchDev& b, const void* plan, const float* scores, int64_t ld, int k, int32_t* S, void* ws,
                 void* stream) {
   if (b.T == 0) return 0;
-  if (b.max_seq_len > kMaxChunks * kChunk) return static_cast<int>(cudaErrorInvalidValue);
+  if (b.max_seq_len > kMaxTopKRow) return static_cast<int>(cudaErrorInvalidValue);
   PlanView pv = plan_view(const_cast<void*>(plan), b.B, b.T);
-  const int cap = b.max_seq_len <= kCacheCap ? ((b.max_seq_len + 3) & ~3) : 0;
-  const size_t smem = sizeof(uint32_t) * (kBins + kCandCap + static_cast<size_t>(cap));
-  auto kern = (cap > 0) ? topk_kernel<1> : topk_kernel<4>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(sizeof(uint32_t) * (kBins + kCandCap + kCacheCap)));
-  if (e != cudaSuccess) return static_cast<int>(e);
-  return static_cast<int>(
-      launch_pdl(kern, dim3(b.T), dim3(kThreads), smem, stream, pv.row_pos, scores, ld, k, S, cap));
+  const int nsl = b.max_seq_len > kSlice ? (b.max_seq_len + kSlice - 1) / kSlice : 1;
+  const int kpad = (k + 3) & ~3;
+  if (nsl > 1 && !ws) return static_cast<int>(cudaErrorInvalidValue);
+  int32_t* cand_ws = static_cast<int32_t*>(ws);
+  const int max_smem = static_cast<int>(sizeof(uint32_t) * (kBins + kCandCap + kSlice));
+  for (auto kern : {topk_kernel<false>, topk_kernel<true>}) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+    if (e != cudaSuccess) return static_cast<int>(e);
+  }
+  const int capA = std::min(kSlice, (b.max_seq_len + 3) & ~3);
+  cudaError_t e = launch_pdl(topk_kernel<false>, dim3(b.T * nsl), dim3(kThreads),
+                             sizeof(uint32_t) * (kBins + kCandCap + static_cast<size_t>(capA)), stream, pv.row_pos,
+                             scores, ld, k, S, cand_ws, nsl, kpad);
+  if (e != cudaSuccess || nsl == 1) return static_cast<int>(e);
+  const int capB = std::min(kSlice, (nsl * k + 3) & ~3);
+  e = launch_pdl(topk_kernel<true>, dim3(b.T), dim3(kThreads),
+                 sizeof(uint32_t) * (kBins + kCandCap + static_cast<size_t>(capB)), stream, pv.row_pos, scores, ld, k,
+                 S, cand_ws, nsl, kpad);
+  return static_cast<int>(e);
 }
 
 }  // namespace dsa

@@ -38,7 +38,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_strings(lib):
-    assert lib.dsa_abi_version() == 1
+    assert lib.dsa_abi_version() == 2
     for s in range(7):
         assert lib.dsa_status_string(s).decode() == dsa.STATUS[s]
     assert lib.dsa_status_string(99).decode() == "unknown status"
@@ -68,7 +68,7 @@ def test_plan_rejects_bad_arguments(lib):
 def test_empty_batch_is_a_no_op(lib):
     b = dsa.DsaBatchC(0, 0, 0, 0, 0, 0, None, None, None)
     assert lib.dsa_index_scores(ctypes.byref(b), None, None, None, None, 64, None, None, None, 0, None) == 0
-    assert lib.dsa_topk(ctypes.byref(b), None, None, 0, 2048, None, None) == 0
+    assert lib.dsa_topk(ctypes.byref(b), None, None, 0, 2048, None, None, 0, None) == 0
     assert lib.dsa_sparse_mla(ctypes.byref(b), None, None, 128, None, None, 2048, 0.07, None, None, None, 0,
                               None) == 0
     assert lib.dsa_layer(ctypes.byref(b), None, None, None, 64, None, None, None, 128, None, 2048, 0.07, None,
@@ -102,13 +102,20 @@ def test_cache_write_validation(lib):
 
 def test_topk_and_mla_validation(lib):
     b = batch()
-    assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE, 384, 0, FAKE, None) == 2
-    assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE, 384, 5000, FAKE, None) == 2
-    assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE, 100, 16, FAKE, None) == 1
-    assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE, 386, 16, FAKE, None) == 1      # ld % 4
-    assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE + 4, 384, 16, FAKE, None) == 1  # misaligned scores
+    assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE, 384, 0, FAKE, None, 0, None) == 2
+    assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE, 384, 5000, FAKE, None, 0, None) == 2
+    assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE, 100, 16, FAKE, None, 0, None) == 1
+    assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE, 386, 16, FAKE, None, 0, None) == 1      # ld % 4
+    assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE + 4, 384, 16, FAKE, None, 0, None) == 1  # misaligned scores
     long_rows = batch(max_seq_len=262145, max_pages=4097)
-    assert lib.dsa_topk(ctypes.byref(long_rows), FAKE, FAKE, 262148, 16, FAKE, None) == 2
+    assert lib.dsa_topk(ctypes.byref(long_rows), FAKE, FAKE, 262148, 16, FAKE, None, 0, None) == 2
+    # rows above 32768 positions need the candidate workspace: T * slices * round4(k) int32
+    sliced = batch(max_seq_len=70000, max_pages=1094, num_pages=2000)
+    need = lib.dsa_topk_workspace_size(ctypes.byref(sliced), 2047)
+    assert need == 4 * 3 * 3 * 2048
+    assert lib.dsa_topk_workspace_size(ctypes.byref(b), 2048) == 0
+    assert lib.dsa_topk(ctypes.byref(sliced), FAKE, FAKE, 70000, 2047, FAKE, None, 0, None) == 1      # no ws
+    assert lib.dsa_topk(ctypes.byref(sliced), FAKE, FAKE, 70000, 2047, FAKE, FAKE, need - 1, None) == 3
     mla = lambda **kw: lib.dsa_sparse_mla(
         ctypes.byref(b), FAKE, kw.get("q", FAKE), kw.get("H", 128), FAKE, FAKE, kw.get("k", 2048),
         kw.get("scale", 0.07), FAKE, None, kw.get("ws", FAKE), kw.get("ws_bytes", 1 << 30), None)
