@@ -17,7 +17,9 @@ Sources ("page" = title of the web page):
   [P5-SWA] same page, section "SWA：让固定窗口沿序列移动": causal visibility C_t = {1..t}.
   [P1-DSA] "MTP 与稀疏注意力：NSA 与 DSA", section "稀疏注意力：NSA 与 DSA": 64 FP8 indexer heads of
            width 128, top 2048, absorbed MLA over a 576-wide latent (512 + 64 rope), per-pair FLOP
-           counts; expanded head width 128 + 64 = 192; k = min(L, 2048).
+           counts; expanded head width 128 + 64 = 192; k = min(L, 2048); for short prefill,
+           DeepSeek-V3.2 emulates DSA with a masked multi-head attention in the expanded form
+           (q.k over 128 + 64 dims and p.v over 128 dims per head).
 
 Readings where the pages leave a step open (each is listed in the design notes):
   * FP8 is OCP e4m3fn; per-token fp32 scales multiply the decoded codes (s^q_t for the query,
@@ -71,6 +73,12 @@ def bf16_decode(bits) -> np.ndarray:
     """Decode bf16 bit patterns (the upper half of an IEEE float32) to float64."""
     b = np.asarray(bits).astype(np.uint16).astype(np.uint32) << np.uint32(16)
     return b.view(np.float32).astype(np.float64)
+
+
+def _values(x) -> np.ndarray:
+    """bf16 bit patterns (uint16 arrays) decoded to float64; float arrays are taken as values."""
+    x = np.asarray(x)
+    return bf16_decode(x) if x.dtype == np.uint16 else x.astype(np.float64)
 
 
 def e4m3_encode(values) -> np.ndarray:
@@ -182,12 +190,12 @@ def sparse_mla_row(t, req, S_t, block_table, q, kv_cache, softmax_scale):
     """
     b = int(req[t])
     sel = np.asarray([j for j in S_t if j >= 0], np.int64)
-    qt = bf16_decode(q[t])                                    # [H, 576]
+    qt = _values(q[t])                                        # [H, 576]
     H = qt.shape[0]
     if sel.size == 0:
         return np.zeros((H, D_V)), np.full(H, -np.inf)
     pages, slots = physical_rows(block_table[b], sel)
-    c = bf16_decode(kv_cache[pages, slots])                   # [|S_t|, 576]
+    c = _values(kv_cache[pages, slots])                       # [|S_t|, 576]
     z = softmax_scale * (qt @ c.T)                            # [H, |S_t|]
     zmax = z.max(axis=1, keepdims=True)
     e = np.exp(z - zmax)
@@ -241,6 +249,53 @@ def cache_write(seq_lens, cu_q, block_table, k_new, c_new_bits, kI_cache, kI_sca
         ks[pages[0], slots[0]] = s
         kv[pages[0], slots[0]] = c_new_bits[t]
     return kI, ks, kv
+
+
+# ---------------------------------------------------------------------------------------------
+# masked MHA mode for short prefill [P1-DSA]: the expanded multi-head form (per head, q and k of
+# width 128 + 64, v of width 128) with the DSA mask of [P5-SA], M = 0 on S_t and -inf elsewhere
+
+def masked_mha_row(t, req, pos, cu_q, seq_lens, S_t, q, k, v, softmax_scale):
+    """Masked MHA of query row t, float64: (o [H, dv], lse [H]).
+
+    Every request is a whole prefill (m_b = n_b): row cu_q[b] + j of k and v holds position j of
+    request b. With K_b, V_b the request's rows,
+        z_h = tau * q_th K_bh^T + M_t,   M_tj = 0 for j in S_t, -inf for every other j < n_b,
+        o_th = softmax(z_h) V_bh,        lse_th = log sum_j exp(z_hj).
+    Entries of S_t below 0 are padding; a position listed twice is still one position of the set.
+    """
+    b, p = int(req[t]), int(pos[t])
+    n = int(seq_lens[b])
+    lo = int(cu_q[b])
+    assert int(cu_q[b + 1]) - lo == n, "masked MHA mode: every request is a whole prefill"
+    sel = np.asarray([j for j in S_t if j >= 0], np.int64)
+    assert np.all(sel <= p), "S_t holds visible positions only"
+    qt = _values(q[t])                                        # [H, dqk]
+    Kb = _values(k[lo:lo + n])                                # [n, H, dqk]
+    Vb = _values(v[lo:lo + n])                                # [n, H, dv]
+    H, dv = qt.shape[0], Vb.shape[2]
+    M = np.full(n, -np.inf)
+    M[sel] = 0.0
+    if sel.size == 0:
+        return np.zeros((H, dv)), np.full(H, -np.inf)
+    z = softmax_scale * np.einsum("hd,jhd->hj", qt, Kb) + M[None, :]   # [H, n]
+    zmax = z.max(axis=1, keepdims=True)
+    e = np.exp(z - zmax)                                      # exp(-inf) = 0 off the mask
+    denom = e.sum(axis=1, keepdims=True)
+    o = np.einsum("hj,jhd->hd", e, Vb) / denom
+    return o, zmax[:, 0] + np.log(denom[:, 0])
+
+
+def masked_mha(seq_lens, cu_q, q, k, v, S, softmax_scale, rows=None):
+    """Output [T, H, dv] and lse [T, H] (float64) of the masked MHA mode for every (or the given) row."""
+    req, pos = query_positions(seq_lens, cu_q)
+    T, H = q.shape[0], q.shape[1]
+    dv = v.shape[2]
+    out = np.zeros((T, H, dv))
+    lse = np.full((T, H), -np.inf)
+    for t in (range(T) if rows is None else rows):
+        out[t], lse[t] = masked_mha_row(t, req, pos, cu_q, seq_lens, S[t], q, k, v, softmax_scale)
+    return out, lse
 
 
 # ---------------------------------------------------------------------------------------------

@@ -263,3 +263,47 @@ def make_batch(wl: Workload, seed: int = 0, extra_pages: int = 0) -> Batch:
     kv_cache = _normal_bf16(rng, (P, PAGE, D_LATENT), chunk_rows=max(1, (1 << 22) // (PAGE * D_LATENT)))
     return Batch(wl, qI, qI_scale, wI, kI_cache, kI_scale, q, kv_cache, block_table,
                  seq_lens, cu_q, needles)
+
+
+# ---------------------------------------------------------------------------------------------
+# inputs of the masked MHA mode for short prefill (expanded heads: q and k of width 128 + 64,
+# v of width 128, one row per position of each whole-prefill request)
+
+D_QK_MHA = 128 + 64
+D_V_MHA = 128
+
+
+@dataclasses.dataclass
+class MhaInputs:
+    """q, k uint16 [T, H, 192] and v uint16 [T, H, 128]: bf16 bits of N(0,1) draws; row cu_q[b] + j
+    of k and v is position j of request b (every request a whole prefill, m_b = n_b)."""
+    q: np.ndarray
+    k: np.ndarray
+    v: np.ndarray
+
+
+def make_mha_inputs(wl: Workload, seed: int = 0) -> MhaInputs:
+    assert tuple(wl.seq_lens) == tuple(wl.q_per_req), "the masked MHA mode takes whole prefills"
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, wl.wid, 7])))
+    T, H = wl.total_q, wl.n_heads
+    rows = max(1, (1 << 22) // (H * D_QK_MHA))
+    q = _normal_bf16(rng, (T, H, D_QK_MHA), chunk_rows=rows)
+    k = _normal_bf16(rng, (T, H, D_QK_MHA), chunk_rows=rows)
+    v = _normal_bf16(rng, (T, H, D_V_MHA), chunk_rows=rows)
+    return MhaInputs(q, k, v)
+
+
+def random_index_sets(seq_lens, q_per_req, k: int, seed: int = 0) -> np.ndarray:
+    """int32 [T, k]: for every query row (request b, position p = n_b - m_b + i) min(k, p + 1)
+    distinct positions drawn uniformly from [0, p], in random order, padded with -1."""
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, 11])))
+    T = int(sum(q_per_req))
+    out = np.full((T, k), -1, np.int32)
+    t = 0
+    for n, m in zip(seq_lens, q_per_req):
+        for i in range(int(m)):
+            p = int(n) - int(m) + i
+            take = min(k, p + 1)
+            out[t, :take] = rng.choice(p + 1, size=take, replace=False) if take < p + 1 else rng.permutation(p + 1)
+            t += 1
+    return out

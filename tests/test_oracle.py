@@ -398,6 +398,106 @@ def test_sparse_mla_shift_invariant_and_order_free():
     np.testing.assert_allclose(l1, l2, rtol=1e-12)
 
 
+# ---------------------------------------------------------------------------------------------
+# masked MHA mode for short prefill: the expanded heads with the DSA mask
+
+def _bf16_values(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).double().numpy()
+
+
+def test_masked_mha_hand_worked():
+    """One head, tau = 1, S_2 = {0, 1}: logits 0 and ln 3 give weights 1/4 and 3/4; position 2 has
+    the largest logit but is not in S_2 and must not count."""
+    q = np.zeros((3, 1, 2))
+    q[2, 0] = [1.0, 0.0]
+    k = np.array([[[0.0, 0.0]], [[math.log(3.0), 0.0]], [[5.0, 0.0]]])
+    v = np.array([[[4.0, 0.0]], [[0.0, 8.0]], [[100.0, 100.0]]])
+    S = np.array([[0, -1], [0, -1], [1, 0]], np.int32)
+    out, lse = O.masked_mha([3], [0, 3], q, k, v, S, 1.0, rows=[2])
+    np.testing.assert_allclose(out[2, 0], [1.0, 6.0], rtol=1e-14)
+    np.testing.assert_allclose(lse[2, 0], math.log(4.0), rtol=1e-14)
+
+
+def test_masked_mha_dense_when_sets_cover_prefix():
+    """With S_t = [0, p] the masked mode is causal multi-head attention (torch SDPA, per request)."""
+    lens, H = [37, 70], 3
+    wl = synth.custom("mha", lens, lens, n_heads=H)
+    x = synth.make_mha_inputs(wl, seed=3)
+    tau = O.default_softmax_scale()
+    cu = [0, lens[0], lens[0] + lens[1]]
+    S = np.full((sum(lens), max(lens)), -1, np.int32)
+    for b, n in enumerate(lens):
+        for i in range(n):
+            S[cu[b] + i, : i + 1] = np.arange(i + 1)
+    out, lse = O.masked_mha(lens, cu, x.q, x.k, x.v, S, tau)
+    q, k, v = (_bf16_values(a) for a in (x.q, x.k, x.v))
+    for b, n in enumerate(lens):
+        sl = slice(cu[b], cu[b] + n)
+        per_head = lambda a: np.ascontiguousarray(a[sl].transpose(1, 0, 2))
+        causal = np.where(np.tril(np.ones((n, n), bool)), 0.0, -np.inf)
+        ref = _sdpa(per_head(q), per_head(k), per_head(v), causal, tau)
+        np.testing.assert_allclose(out[sl], ref.transpose(1, 0, 2), rtol=1e-10, atol=1e-12)
+        logits = tau * np.einsum("thd,jhd->thj", q[sl], k[sl]) + causal[:, None, :]
+        np.testing.assert_allclose(lse[sl], torch.logsumexp(torch.from_numpy(logits), -1).numpy(), rtol=1e-12)
+
+
+def test_masked_mha_emulates_absorbed_sparse_mla():
+    """The masked MHA mode computes DSA: with k_jh = [W_UK_h c_j[:512], c_j[512:]], v_jh = W_UV_h c_j[:512]
+    and the absorbed query [W_UK_h^T q_nope, q_rope], its output is the absorbed sparse MLA's output
+    mapped by W_UV_h, on the same S_t (sparse sets, several heads, a ragged two-request batch)."""
+    lens, H, kk = [50, 81], 3, 13
+    wl = synth.custom("mha_vs_mla", lens, lens, n_heads_index=2, topk=kk, n_heads=H)
+    bt = synth.make_batch(wl, seed=5, extra_pages=2)
+    rng = np.random.default_rng(9)
+    T = sum(lens)
+    W_uk = rng.standard_normal((H, 128, 512)) / math.sqrt(512)
+    W_uv = rng.standard_normal((H, 128, 512)) / math.sqrt(512)
+    q_nope = rng.standard_normal((T, H, 128))
+    q_rope = rng.standard_normal((T, H, 64))
+    req, pos = O.query_positions(bt.seq_lens, bt.cu_q)
+    c = np.zeros((T, 576))                      # latent row of every (request, position) = query row
+    for t in range(T):
+        c[t] = _latent_rows(bt, int(req[t]), int(pos[t]) + 1)[int(pos[t])]
+    k_mha = np.concatenate([np.einsum("hde,te->thd", W_uk, c[:, :512]),
+                            np.broadcast_to(c[:, None, 512:], (T, H, 64))], axis=2)
+    v_mha = np.einsum("hde,te->thd", W_uv, c[:, :512])
+    q_mha = np.concatenate([q_nope, q_rope], axis=2)
+    q_abs = np.concatenate([np.einsum("hde,thd->the", W_uk, q_nope), q_rope], axis=2)
+    S = synth.random_index_sets(lens, lens, kk, seed=2)
+    tau = O.default_softmax_scale()
+    o_mha, lse_mha = O.masked_mha(bt.seq_lens, bt.cu_q, q_mha, k_mha, v_mha, S, tau)
+    o_mla, lse_mla = O.sparse_mla(bt.seq_lens, bt.cu_q, bt.block_table, q_abs, bt.kv_cache, S, tau)
+    np.testing.assert_allclose(o_mha, np.einsum("hde,the->thd", W_uv, o_mla), rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(lse_mha, lse_mla, rtol=1e-12, atol=1e-12)
+
+
+def test_masked_mha_single_position_and_set_semantics():
+    lens, H = [40], 2
+    wl = synth.custom("mha1", lens, lens, n_heads=H)
+    x = synth.make_mha_inputs(wl, seed=4)
+    S = np.full((40, 6), -1, np.int32)
+    S[:, 0] = 0
+    out, _ = O.masked_mha(lens, [0, 40], x.q, x.k, x.v, S, 0.1)
+    v = _bf16_values(x.v)
+    for t in range(40):
+        assert np.array_equal(out[t], v[0])
+    S2 = synth.random_index_sets(lens, lens, 5, seed=1)
+    dup = np.concatenate([S2, S2[:, :1]], axis=1)  # a position listed twice counts once
+    o1, l1 = O.masked_mha(lens, [0, 40], x.q, x.k, x.v, S2, 0.1)
+    o2, l2 = O.masked_mha(lens, [0, 40], x.q, x.k, x.v, dup, 0.1)
+    np.testing.assert_allclose(o1, o2, rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(l1, l2, rtol=1e-14)
+
+
+def test_random_index_sets_are_valid():
+    S = synth.random_index_sets([300, 5], [300, 2], 64, seed=0)
+    _, pos = O.query_positions([300, 5], [0, 300, 302])
+    for t in range(S.shape[0]):
+        sel = S[t][S[t] >= 0]
+        assert sel.size == min(64, pos[t] + 1) and np.unique(sel).size == sel.size
+        assert sel.max() <= pos[t] and np.all(S[t][sel.size:] == -1)
+
+
 def test_softmax_scale_reading():
     assert O.default_softmax_scale() == 1.0 / math.sqrt(192.0)
 
@@ -410,6 +510,8 @@ def test_cost_model_matches_printed_table(golden_dir):
     assert round(CM.pair_flops_mla_absorbed() / 1e3) == g["pair_flops_mla_k"]
     assert round(CM.pair_flops_indexer() / 1e3) == g["pair_flops_indexer_k"]
     assert round(100 * CM.bytes_per_token_index() / CM.bytes_per_token_latent()) == g["index_cache_overhead_pct"]
+    assert round(CM.pair_flops_mha_expanded() / 1e3) == g["pair_flops_mha_expanded_k"]
+    assert round(CM.pair_flops_mla_absorbed() / CM.pair_flops_mha_expanded(), 1) == g["absorbed_over_expanded"]
     for row in g["rows"]:
         dec, rd, pre = CM.per_layer_costs(row["L"])
         assert [round(x / 1e9, 2) for x in dec] == row["decode_gflops"]
