@@ -17,7 +17,10 @@ The JSON line also carries
   e2e           the same metric through the public API with host (pinned) inputs: per step the
                 queries and batch metadata go host->device and the output comes back; the paged
                 caches stay resident (they are the cache, not per-step inputs);
-  cpu_baseline  the CPU oracle (float64 numpy) timed on this host on a bounded sample of rows.
+  cpu_baseline  the CPU oracle (float64 numpy) timed on this host on a bounded sample of rows;
+  short_prefill the masked MHA mode (the dense fallback for short prefill) on its own shape,
+                L = 2048, 16 heads, k = 512: mask + attention kernels, event-timed, in TFLOP/s
+                of the dense causal work against the measured bf16 peak.
 `--impl reference` times that oracle alone as the reference arm.
 """
 from __future__ import annotations
@@ -186,6 +189,42 @@ class ClockSampler:
 # ---------------------------------------------------------------------------------------------
 # oracle timing (CPU baseline / reference arm)
 
+def short_prefill_mha(dev, timed_mean, n, tf_peak):
+    """The masked MHA mode (expanded heads, the DSA mask) on the short-prefill shape: one request
+    of 2048 positions, 16 heads, k = 512. The index sets are random valid sets (the dense tiles'
+    work does not depend on which positions are selected). Algorithmic work: the causal pairs
+    L(L+1)/2 times 2H(192 + 128) FLOPs."""
+    import torch
+    import sparse_attention_12_b200 as dsa
+    from sparse_attention_12_b200 import synth
+    wl = synth.workload("prefill_2048")
+    L, H, k = int(wl.seq_lens[0]), wl.n_heads, wl.topk
+    x = synth.make_mha_inputs(wl, seed=0)
+    S = torch.from_numpy(synth.random_index_sets(wl.seq_lens, wl.q_per_req, k, seed=0)).to(dev)
+    i32 = lambda v: torch.tensor(v, dtype=torch.int32, device=dev)
+    bt = torch.arange((L + 63) // 64, dtype=torch.int32, device=dev)[None].contiguous()
+    batch = dsa.Batch(i32([L]), i32([0, L]), bt, int(bt.shape[1]), L, L, L)
+    plan = dsa.plan(batch, 16)
+    bf = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    q, kk, v = bf(x.q), bf(x.k), bf(x.v)
+    out = torch.empty((L, H, 128), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(16, dsa.load().dsa_masked_mha_workspace_size(batch.ref(), H, k)), dtype=torch.uint8,
+                     device=dev)
+    fn = lambda: dsa.masked_mha(batch, plan, q, kk, v, S, wl.softmax_scale, out=out, ws=ws)
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    status = dsa.status_read(plan)
+    if status != 0:
+        raise RuntimeError(f"device status {status} in the masked MHA mode")
+    ms = timed_mean(fn, n)
+    flops = L * (L + 1) / 2 * 2 * H * (192 + 128)
+    tf = flops / (ms / 1e3) / 1e12
+    return {"workload": "prefill_2048 (masked MHA mode)", "us": 1e3 * ms, "algorithmic_flops": flops,
+            "TFLOPs": tf, "peak_TFLOPs": tf_peak, "frac": tf / tf_peak, "launches": 2,
+            "note": "mask kernel + attention kernel, one call, event-timed; random valid index sets"}
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -229,6 +268,7 @@ def main():
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-short-prefill", action="store_true")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -391,6 +431,10 @@ def main():
                                                db.kv_cache), max(3, min(args.steps, 20)))
     cw_bytes = T * (128 * 4 + 576 * 2 + 128 + 4 + 576 * 2)
 
+    short = None
+    if not args.no_short_prefill:
+        short = short_prefill_mha(dev, timed_mean, max(3, min(args.steps, 20)), tf_peak)
+
     # end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -462,6 +506,7 @@ def main():
         "stages": stage_report,
         "cache_write": {"us": 1e3 * cw_ms, "GBps": cw_bytes / (cw_ms / 1e3) / 1e9, "algorithmic_bytes": cw_bytes,
                         "note": "the step before the layer, not in the step; one launch, event-timed"},
+        "short_prefill": short,
         "e2e": e2e,
         "cpu_baseline": cpu,
         "gpu_launches": launches_per_step * args.steps,

@@ -46,11 +46,13 @@
 extern "C" {
 #endif
 
-#define DSA_ABI_VERSION 2
+#define DSA_ABI_VERSION 3
 #define DSA_PAGE_SIZE 64   /* positions per cache page */
 #define DSA_D_INDEX 128    /* indexer head width d_h^I */
 #define DSA_D_LATENT 576   /* latent width: 512 + 64 rope */
 #define DSA_D_V 512        /* value width: first 512 latent dims */
+#define DSA_D_QK_MHA 192   /* masked MHA mode: expanded q/k head width, 128 + 64 rope */
+#define DSA_D_V_MHA 128    /* masked MHA mode: expanded v head width */
 
 typedef enum {
   DSA_OK = 0,
@@ -139,6 +141,31 @@ dsa_status_t dsa_topk(const dsa_batch_t* batch, const void* plan, const float* s
 size_t dsa_sparse_mla_workspace_size(const dsa_batch_t* batch, int H, int k);
 dsa_status_t dsa_sparse_mla(const dsa_batch_t* batch, const void* plan, const void* q, int H,
                             const void* kv_cache, const int32_t* S, int k, float softmax_scale, void* out,
+                            float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- masked MHA mode for short prefill (an alternative to step 3) -------------------------
+ * "MTP 与稀疏注意力：NSA 与 DSA", section "稀疏注意力：NSA 与 DSA": in a short prefill the absorbed
+ * form costs 2H(512+64) + 2H*512 FLOPs per (query, key) pair against 2H(128+64) + 2H*128 for the
+ * expanded multi-head form, so DeepSeek-V3.2 emulates DSA there with a masked multi-head attention.
+ * The mask is the DSA mask of "DeepSeek Sparse Attention：从 SWA 到稀疏 Attention 计算", section
+ * "Sparse Attention": M_tj = 0 for j in S_t, -inf elsewhere. For query row t and head h:
+ *     out[t][h] = sum_j softmax_j(scale * q[t][h] . k[j][h] + M_tj) v[j][h]
+ * Every request must be a whole prefill (m_b = n_b): row cu_q[b] + j of k and v holds position j of
+ * request b. A request with n_b != m_b is recorded as DSA_ERR_DEVICE_INDEX and its rows are not
+ * written.
+ * q, k     bf16 [T, H, 192]   expanded queries and keys (128 "nope" + 64 rope dims per head)
+ * v        bf16 [T, H, 128]   expanded values
+ * S        int32 [T, topk]    index sets as dsa_topk writes them (entries < 0 skipped; a position
+ *                             listed twice counts once; an entry above the row's position is
+ *                             recorded as DSA_ERR_DEVICE_INDEX and skipped)
+ * out      bf16 [T, H, 128]   lse f32 [T, H] or NULL (natural log; -inf for an empty set)
+ * 1 <= H <= 128, 1 <= topk <= 4096, max_seq_len <= 65536. The plan must be made for this batch.
+ * ws/ws_bytes: dsa_masked_mha_workspace_size bytes (the bitmap of S_t, T * max_seq_len / 8 bytes
+ * rounded up). Dense tiles of 128 queries x 128 keys over each query tile's causal range, tcgen05
+ * MMAs with S, P and O in TMEM. */
+size_t dsa_masked_mha_workspace_size(const dsa_batch_t* batch, int H, int topk);
+dsa_status_t dsa_masked_mha(const dsa_batch_t* batch, const void* plan, const void* q, const void* k,
+                            const void* v, int H, const int32_t* S, int topk, float softmax_scale, void* out,
                             float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /* ---- the whole path ---------------------------------------------------------------------

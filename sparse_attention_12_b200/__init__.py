@@ -19,6 +19,8 @@ PAGE_SIZE = 64
 D_INDEX = 128
 D_LATENT = 576
 D_V = 512
+D_QK_MHA = 192
+D_V_MHA = 128
 
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported size", 3: "workspace too small", 4: "CUDA error",
           5: "a kernel wait timed out", 6: "a kernel met an out-of-range index"}
@@ -38,7 +40,8 @@ class DsaBatchC(ctypes.Structure):
 
 EXPORTS = ("dsa_abi_version", "dsa_status_string", "dsa_plan_workspace_size", "dsa_plan", "dsa_status_read",
            "dsa_index_scores", "dsa_topk_workspace_size", "dsa_topk", "dsa_sparse_mla_workspace_size", "dsa_sparse_mla",
-           "dsa_layer_workspace_size", "dsa_layer", "dsa_layer_noalloc", "dsa_cache_write")
+           "dsa_layer_workspace_size", "dsa_layer", "dsa_layer_noalloc", "dsa_cache_write",
+           "dsa_masked_mha_workspace_size", "dsa_masked_mha")
 
 _lib = None
 
@@ -68,6 +71,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "dsa_layer": (I, [BP, P, P, P, I, P, P, P, I, P, I, ctypes.c_float, P, P, P, P, SZ, P]),
         "dsa_layer_noalloc": (I, [BP, P, P, P, I, P, P, P, I, P, I, ctypes.c_float, P, P, P, P]),
         "dsa_cache_write": (I, [BP, P, P, P, P, P, P, P]),
+        "dsa_masked_mha_workspace_size": (SZ, [BP, I, I]),
+        "dsa_masked_mha": (I, [BP, P, P, P, P, I, P, I, ctypes.c_float, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -219,6 +224,31 @@ def sparse_mla(batch: Batch, plan_ws, q, kv_cache, S, softmax_scale: float, out=
     _check(lib.dsa_sparse_mla(batch.ref(), plan_ws.data_ptr(), q.data_ptr(), H, kv_cache.data_ptr(), S.data_ptr(),
                               k, float(softmax_scale), out.data_ptr(), _ptr(lse), _ptr(ws),
                               0 if ws is None else ws.numel(), _stream()), "dsa_sparse_mla")
+    return out
+
+
+def masked_mha(batch: Batch, plan_ws, q, k, v, S, softmax_scale: float, out=None, lse=None, ws=None):
+    """Masked MHA mode for short prefill (dsa_masked_mha): expanded q, k [T, H, 192] and v [T, H, 128]
+    (bf16, every request a whole prefill), index sets S [T, topk]. Returns out [T, H, 128] bf16."""
+    T = batch.total_q
+    H = int(q.shape[1])
+    topk = int(S.shape[1])
+    _need(q, "q", torch.bfloat16, (T, H, D_QK_MHA))
+    _need(k, "k", torch.bfloat16, (T, H, D_QK_MHA))
+    _need(v, "v", torch.bfloat16, (T, H, D_V_MHA))
+    _need(S, "S", torch.int32, (T, topk))
+    lib = load()
+    if out is None:
+        out = torch.empty((T, H, D_V_MHA), dtype=torch.bfloat16, device="cuda")
+    _need(out, "out", torch.bfloat16, (T, H, D_V_MHA))
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (T, H))
+    need = lib.dsa_masked_mha_workspace_size(batch.ref(), H, topk)
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device="cuda")
+    _check(lib.dsa_masked_mha(batch.ref(), plan_ws.data_ptr(), q.data_ptr(), k.data_ptr(), v.data_ptr(), H,
+                              S.data_ptr(), topk, float(softmax_scale), out.data_ptr(), _ptr(lse), ws.data_ptr(),
+                              ws.numel(), _stream()), "dsa_masked_mha")
     return out
 
 

@@ -167,6 +167,30 @@ dsa_status_t dsa_cache_write(const dsa_batch_t* batch, const void* plan, const f
   return from_cuda(launch_cache_write(to_dev(batch), plan, k_new, c_new, kI_cache, kI_scale, kv_cache, stream));
 }
 
+size_t dsa_masked_mha_workspace_size(const dsa_batch_t* batch, int H, int topk) {
+  if (check_batch(batch) != DSA_OK || H < 1 || H > 128 || topk < 1 || topk > kMaxTopK ||
+      batch->max_seq_len > kMaxMhaSeqLen)
+    return 0;
+  return masked_mha_ws_bytes(batch->total_q, batch->max_seq_len);
+}
+
+dsa_status_t dsa_masked_mha(const dsa_batch_t* batch, const void* plan, const void* q, const void* k, const void* v,
+                            int H, const int32_t* S, int topk, float softmax_scale, void* out, float* lse, void* ws,
+                            size_t ws_bytes, void* stream) {
+  dsa_status_t st = check_batch(batch);
+  if (st != DSA_OK) return st;
+  if (H < 1 || H > 128 || topk < 1 || topk > kMaxTopK) return DSA_ERR_UNSUPPORTED;
+  if (batch->total_q == 0) return DSA_OK;
+  if (batch->max_seq_len > kMaxMhaSeqLen || batch->num_requests > 65535) return DSA_ERR_UNSUPPORTED;
+  if (!plan || !q || !k || !v || !S || !out || !ws) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(plan) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(ws))
+    return DSA_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || softmax_scale != softmax_scale) return DSA_ERR_INVALID_ARG;
+  if (ws_bytes < masked_mha_ws_bytes(batch->total_q, batch->max_seq_len)) return DSA_ERR_WORKSPACE;
+  return from_cuda(
+      launch_masked_mha(to_dev(batch), plan, q, k, v, H, S, topk, softmax_scale, out, lse, ws, stream));
+}
+
 size_t dsa_layer_workspace_size(const dsa_batch_t* batch, int nhI, int H, int k) {
   if (check_batch(batch) != DSA_OK || !valid_nhI(nhI) || H < 1 || H > 128 || k < 1 || k > kMaxTopK) return 0;
   const size_t T = static_cast<size_t>(batch->total_q);

@@ -38,7 +38,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_strings(lib):
-    assert lib.dsa_abi_version() == 2
+    assert lib.dsa_abi_version() == 3
     for s in range(7):
         assert lib.dsa_status_string(s).decode() == dsa.STATUS[s]
     assert lib.dsa_status_string(99).decode() == "unknown status"
@@ -142,3 +142,29 @@ def test_layer_workspace_accounting(lib):
     args = [ctypes.byref(b), FAKE, FAKE, FAKE, 64, FAKE, FAKE, FAKE, 128, FAKE, 2048, 0.07, FAKE, None, None, FAKE]
     assert lib.dsa_layer(*args, n - 1, None) == 3
     assert lib.dsa_layer(*args[:4], 40, *args[5:], n, None) == 2
+
+
+def test_masked_mha_validation(lib):
+    b = batch()
+    need = lib.dsa_masked_mha_workspace_size(ctypes.byref(b), 16, 512)
+    assert need == 4 * 3 * 12            # one bit per position: 300 positions -> 3 tiles of 4 words per row
+    call = lambda **kw: lib.dsa_masked_mha(
+        ctypes.byref(kw.get("b", b)), kw.get("plan", FAKE), kw.get("q", FAKE), kw.get("k", FAKE), kw.get("v", FAKE),
+        kw.get("H", 16), kw.get("S", FAKE), kw.get("topk", 512), kw.get("scale", 0.07), kw.get("out", FAKE), None,
+        kw.get("ws", FAKE), kw.get("ws_bytes", need), None)
+    assert call(H=0) == 2
+    assert call(H=129) == 2
+    assert call(topk=0) == 2
+    assert call(topk=4097) == 2
+    assert call(v=None) == 1
+    assert call(S=None) == 1
+    assert call(k=FAKE + 2) == 1        # misaligned
+    assert call(scale=-1.0) == 1
+    assert call(ws=None) == 1
+    assert call(ws_bytes=need - 1) == 3
+    long_req = batch(max_seq_len=65537, max_pages=1025, num_pages=2000)
+    assert call(b=long_req) == 2
+    assert lib.dsa_masked_mha_workspace_size(ctypes.byref(long_req), 16, 512) == 0
+    empty = dsa.DsaBatchC(0, 0, 0, 0, 0, 0, None, None, None)
+    assert lib.dsa_masked_mha(ctypes.byref(empty), None, None, None, None, 16, None, 512, 0.07, None, None, None, 0,
+                              None) == 0
