@@ -13,23 +13,28 @@
 //
 // Two kernels:
 //   * mha_mask_kernel: the bitmap of S_t, one row of 32-bit words per query row (bit j of word w is
-//     position 32w + j), built in shared memory with atomics, then stored with 16-byte stores.
+//     position 32w + j), one warp per row, built in shared memory with atomics, then stored with
+//     16-byte stores.
 //   * masked_mha_kernel: one CTA per (head, 128-query tile, request), a flash-attention pass over the
 //     key tiles 0 .. the tile's last position (causal by construction: S_t only holds j <= t).
-//       - warp 0: TMA producer. Q (3 boxes of 128 rows x 64 dims, 128-byte swizzle) once, then per
-//         key tile K (3 boxes) and V (2 boxes) into two-stage rings.
+//       - warp 0: TMA producers. Lane 0: Q (3 boxes of 128 rows x 64 dims, 128-byte swizzle) once,
+//         then K (3 boxes per key tile) into a two-stage ring; lane 1: V (2 boxes per key tile) into
+//         its own two-stage ring.
 //       - warp 1: TMEM allocator and the single MMA-issuing thread. S = Q K^T is 12 tcgen05.mma
 //         (M = 128 queries, N = 128 keys, K = 16) from shared memory into one of two S buffers in
 //         TMEM; O += P V is 8 tcgen05.mma with P read from TMEM (the A operand) and V from shared
 //         memory (MN-major), into O in TMEM. Order: S0, S1, then P V(i), S(i+2) per tile.
-//       - warps 2..9: softmax, two warps per TMEM lane quadrant (thread = query row, 64 keys each).
-//         They mask with the bitmap, keep an online softmax whose reference maximum moves only when
-//         a tile's maximum exceeds it by more than 2^8 (then they rescale their half of O's row),
-//         and write bf16 P into TMEM (two buffers). At the end they normalise O and store bf16 rows.
+//       - warps 2..9: softmax, two warps per TMEM lane quadrant (thread = query row, 64 keys each;
+//         four warps of 32 keys measured slower: the per-tile exchange and waits outweigh the extra
+//         latency hiding). They mask with the bitmap, keep an online softmax whose reference maximum
+//         moves only when a tile's maximum exceeds it by more than 2^8 (then they rescale their half
+//         of O's row), and write bf16 P into TMEM (two buffers). At the end they normalise O and
+//         store bf16 rows.
 //   TMEM: S at columns 0 and 128, O at 256, P at 384 and 448 (bf16 pairs): all 512 columns.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 
 #include "dsa_internal.h"
@@ -51,7 +56,10 @@ constexpr int kVBlks = kDvh / 64;      // 2
 constexpr int kStages = 2;             // K and V ring depth
 constexpr int kSoftWarp0 = 2;
 constexpr int kSoftWarps = 8;
-constexpr int kSubs = kSoftWarps / 4;  // column halves per lane quadrant
+constexpr int kSubs = kSoftWarps / 4;  // softmax warps per TMEM lane quadrant
+constexpr int kCols = kTile / kSubs;   // keys of a tile per softmax warp (64)
+constexpr int kWords = kCols / 32;     // mask words (and 32-column TMEM loads) per softmax warp and tile
+constexpr int kOCols = kDvh / kSubs;   // O columns per softmax warp (64)
 constexpr int kThreads = 32 * (kSoftWarp0 + kSoftWarps);
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -73,7 +81,7 @@ struct Smem {
 };
 static_assert(Smem::kDynamic <= 232448, "masked MHA shared memory exceeds the 227 KB limit");
 static_assert(kDqk % 64 == 0 && kDvh % 64 == 0, "head widths in 64-dim blocks");
-static_assert(kTile == 32 * 2 * kSubs, "softmax warps cover a tile");
+static_assert(kCols % 32 == 0 && kOCols % 32 == 0, "softmax warps work in 32-column TMEM loads");
 
 enum : int {
   B_QFULL = 0,                 // 1    TMA bytes of Q
@@ -112,31 +120,45 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
 }
 
 // Bitmap of S_t for every query row: bit (j & 31) of word j / 32 set for j in S_t. Entries below 0
-// are padding; an entry above the row's position is reported and skipped.
+// are padding; an entry above the row's position is reported and skipped. One warp per row, each
+// warp with its own ldw words of shared memory (no block-wide synchronisation).
 __global__ void __launch_bounds__(256) mha_mask_kernel(const int32_t* __restrict__ row_pos,
-                                                       const int32_t* __restrict__ S, int k, int ldw,
+                                                       const int32_t* __restrict__ S, int k, int ldw, int T,
                                                        uint32_t* __restrict__ mask, uint32_t* status) {
   extern __shared__ uint32_t words[];
   pdl_trigger();
   pdl_wait();  // S_t and the plan come from earlier kernels
-  const int t = blockIdx.x;
-  for (int w = threadIdx.x; w < ldw; w += blockDim.x) words[w] = 0u;
-  __syncthreads();
+  const int rows = static_cast<int>(blockDim.x >> 5);
+  const int warp = warp_id(), lane = lane_id();
+  const int t = blockIdx.x * rows + warp;
+  if (t >= T) return;
+  uint32_t* wrow = words + warp * ldw;
+  for (int w = lane; w < ldw; w += 32) wrow[w] = 0u;
+  __syncwarp();
   const int p = __ldg(row_pos + t);
   const int32_t* St = S + static_cast<int64_t>(t) * k;
-  for (int e = threadIdx.x; e < k; e += blockDim.x) {
-    const int j = __ldg(St + e);
-    if (j < 0) continue;
-    if (j > p || j >= 32 * ldw) {
-      report_error(status, kDevErrIndex);
-      continue;
+  for (int e0 = 0; e0 < k; e0 += 32 * 8) {
+    int jv[8];  // eight loads in flight per lane before the first atomic
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = e0 + 32 * u + lane;
+      jv[u] = (e < k) ? __ldg(St + e) : -1;
     }
-    atomicOr(&words[j >> 5], 1u << (j & 31));
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = jv[u];
+      if (j < 0) continue;
+      if (j > p || j >= 32 * ldw) {
+        report_error(status, kDevErrIndex);
+        continue;
+      }
+      atomicOr(&wrow[j >> 5], 1u << (j & 31));
+    }
   }
-  __syncthreads();
+  __syncwarp();
   uint4* dst = reinterpret_cast<uint4*>(mask + static_cast<int64_t>(t) * ldw);
-  for (int w4 = threadIdx.x; w4 < ldw / 4; w4 += blockDim.x)
-    dst[w4] = make_uint4(words[4 * w4], words[4 * w4 + 1], words[4 * w4 + 2], words[4 * w4 + 3]);
+  for (int w4 = lane; w4 < ldw / 4; w4 += 32)
+    dst[w4] = make_uint4(wrow[4 * w4], wrow[4 * w4 + 1], wrow[4 * w4 + 2], wrow[4 * w4 + 3]);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -195,35 +217,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ---------- TMA producer ----------
-    if (lane == 0 && nkt > 0) {
-      mbar_arrive_expect_tx(&bar[B_QFULL], kQBlks * kBlk);
-      for (int blk = 0; blk < kQBlks; ++blk)
-        tma_load_3d(base + Smem::kQ + blk * kBlk, &qmap, 64 * blk, h, row0 + q0, &bar[B_QFULL]);
+    // ---------- TMA producers: lane 0 Q and the K ring, lane 1 the V ring ----------
+    // (independent loops: K(i+2) goes out as soon as S(i) has consumed its stage, without waiting
+    // behind V(i+1), whose stage frees only after P V(i-1))
+    if (lane < 2 && nkt > 0) {
+      const bool is_k = lane == 0;
+      const int nblk = is_k ? kQBlks : kVBlks;
+      const CUtensorMap* map = is_k ? &kmap : &vmap;
+      uint8_t* ring = base + (is_k ? Smem::kK : Smem::kV);
+      uint64_t* full = &bar[is_k ? B_KFULL : B_VFULL];
+      uint64_t* empty = &bar[is_k ? B_KEMPTY : B_VEMPTY];
+      if (is_k) {
+        mbar_arrive_expect_tx(&bar[B_QFULL], kQBlks * kBlk);
+        for (int blk = 0; blk < kQBlks; ++blk)
+          tma_load_3d(base + Smem::kQ + blk * kBlk, &qmap, 64 * blk, h, row0 + q0, &bar[B_QFULL]);
+      }
       bool ok = true;
       for (int i = 0; i < nkt && ok; ++i) {
         const int s = i & 1;
-        const uint32_t par = ((i >> 1) & 1) ^ 1;
-        ok = mbar_wait(&bar[B_KEMPTY + s], par, p.status, kDevErrTimeout);
+        ok = mbar_wait(&empty[s], ((i >> 1) & 1) ^ 1, p.status, kDevErrTimeout);
         if (!ok) break;
-        mbar_arrive_expect_tx(&bar[B_KFULL + s], kQBlks * kBlk);
-        for (int blk = 0; blk < kQBlks; ++blk)
-          tma_load_3d(base + Smem::kK + (s * kQBlks + blk) * kBlk, &kmap, 64 * blk, h, row0 + i * kTile,
-                      &bar[B_KFULL + s]);
-        ok = mbar_wait(&bar[B_VEMPTY + s], par, p.status, kDevErrTimeout);
-        if (!ok) break;
-        mbar_arrive_expect_tx(&bar[B_VFULL + s], kVBlks * kBlk);
-        for (int blk = 0; blk < kVBlks; ++blk)
-          tma_load_3d(base + Smem::kV + (s * kVBlks + blk) * kBlk, &vmap, 64 * blk, h, row0 + i * kTile,
-                      &bar[B_VFULL + s]);
+        mbar_arrive_expect_tx(&full[s], nblk * kBlk);
+        for (int blk = 0; blk < nblk; ++blk)
+          tma_load_3d(ring + (s * nblk + blk) * kBlk, map, 64 * blk, h, row0 + i * kTile, &full[s]);
       }
       // no copy may still be landing when the CTA exits
-      mbar_wait(&bar[B_QFULL], 0, p.status, kDevErrTimeout);
+      if (is_k) mbar_wait(&bar[B_QFULL], 0, p.status, kDevErrTimeout);
       if (ok)
-        for (int i = max(0, nkt - kStages); i < nkt; ++i) {
-          mbar_wait(&bar[B_KFULL + (i & 1)], (i >> 1) & 1, p.status, kDevErrTimeout);
-          mbar_wait(&bar[B_VFULL + (i & 1)], (i >> 1) & 1, p.status, kDevErrTimeout);
-        }
+        for (int i = max(0, nkt - kStages); i < nkt; ++i)
+          mbar_wait(&full[i & 1], (i >> 1) & 1, p.status, kDevErrTimeout);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -275,36 +297,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ---------- softmax + epilogue (warps 2..9: thread = query row r, keys 64*sub .. 64*sub+63) ----------
+    // ---------- softmax + epilogue (warps 2..9: thread = query row r, keys kCols*sub .. +kCols-1) ----------
     const int quad = warp & 3;
     const int sub = (warp - kSoftWarp0) >> 2;
     const int r = quad * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const bool row_ok = r < nrows;
     const int64_t t = static_cast<int64_t>(row0) + q0 + r;
-    const uint2* mrow = reinterpret_cast<const uint2*>(p.mask + (row_ok ? t : 0) * p.ldw) + sub;
+    // words 4i + kWords*sub .. + kWords-1 cover this warp's keys of tile i
+    const uint32_t* mrow = p.mask + (row_ok ? t : 0) * p.ldw + kWords * sub;
     float* red = reinterpret_cast<float*>(base + Smem::kRed);
     float* redl = reinterpret_cast<float*>(base + Smem::kRedL);
     const float sl2 = p.scale_log2;
     float m_ref = -INFINITY, l = 0.f, lr = 0.f;
     bool ok = true;
-    uint2 mk = (row_ok && nkt > 0) ? __ldg(mrow) : make_uint2(0u, 0u);
+    uint32_t mk[kWords], mk_next[kWords];
+#pragma unroll
+    for (int w = 0; w < kWords; ++w) mk[w] = (row_ok && nkt > 0) ? __ldg(mrow + w) : 0u;
     for (int i = 0; i < nkt && ok; ++i) {
       const int s = i & 1;
-      const uint2 mk_next = (row_ok && i + 1 < nkt) ? __ldg(mrow + 2 * (i + 1)) : make_uint2(0u, 0u);
+#pragma unroll
+      for (int w = 0; w < kWords; ++w) mk_next[w] = (row_ok && i + 1 < nkt) ? __ldg(mrow + 4 * (i + 1) + w) : 0u;
       ok = __all_sync(0xffffffffu, mbar_wait(&bar[B_SFULL + s], (i >> 1) & 1, p.status, kDevErrTimeout));
       if (!ok) break;
       tc_fence_after();
-      const uint32_t srow = tmem + lane_base + kColS + kTile * s + 64 * sub;
-      uint32_t v0[32], v1[32];
-      tmem_ld32_sync(srow, v0);
-      tmem_ld32_sync(srow + 32, v1);
-      float pmax = -INFINITY;
+      // this warp's kCols scores of the row, -inf where the position is not in S_t
+      float x[kCols];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        if ((mk.x >> j) & 1u) pmax = fmaxf(pmax, __uint_as_float(v0[j]));
-        if ((mk.y >> j) & 1u) pmax = fmaxf(pmax, __uint_as_float(v1[j]));
+      for (int w = 0; w < kWords; ++w) {
+        uint32_t v[32];
+        tmem_ld32_sync(tmem + lane_base + kColS + kTile * s + kCols * sub + 32 * w, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[32 * w + j] = ((mk[w] >> j) & 1u) ? __uint_as_float(v[j]) : -INFINITY;
       }
+      // maximum as a tree (short dependency chains)
+      static_assert(kCols == 64, "the tree below covers 64 scores");
+      float mx[8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+        mx[a] = fmaxf(fmaxf(fmaxf(x[a], x[a + 8]), fmaxf(x[a + 16], x[a + 24])),
+                      fmaxf(fmaxf(x[a + 32], x[a + 40]), fmaxf(x[a + 48], x[a + 56])));
+      float pmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       pmax *= sl2;  // positive scale: the maximum commutes with it (-inf stays -inf)
       red[(s * kSubs + sub) * 128 + r] = pmax;
       __syncwarp();
@@ -322,15 +355,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_ref = tmax;
       }
       if (__any_sync(0xffffffffu, need && i > 0)) {
-        // rescale this warp's half of the O rows once P V(i-1) has landed (rows without a new
+        // rescale this warp's part of the O rows once P V(i-1) has landed (rows without a new
         // reference maximum multiply by 1)
         ok = __all_sync(0xffffffffu,
                         mbar_wait(&bar[B_PVDONE + ((i - 1) & 1)], ((i - 1) >> 1) & 1, p.status, kDevErrTimeout));
         if (!ok) break;
         tc_fence_after();
-        const uint32_t ocol = tmem + lane_base + kColO + 64 * sub;
+        const uint32_t ocol = tmem + lane_base + kColO + kOCols * sub;
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < kOCols / 32; ++c) {
           uint32_t o[32];
           tmem_ld32_sync(ocol + 32 * c, o);
 #pragma unroll
@@ -346,31 +379,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
       }
       const float m_use = (m_ref > -INFINITY) ? m_ref : 0.f;  // m_ref = -inf: every key so far masked
-      uint32_t pk[32];
+      // p = 2^(scale' x - m): masked entries give 2^-inf = 0. Sums on four independent accumulators:
+      // l of the fp32 weights (for the log-sum-exp), lr of the bf16-rounded weights the MMA uses.
+      uint32_t pk[kCols / 2];
+      float la[4] = {0.f, 0.f, 0.f, 0.f}, lra[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j2 = 0; j2 < 16; ++j2) {
-        const int j = 2 * j2;
-        const float a0 = ((mk.x >> j) & 1u) ? fast_exp2(fmaf(__uint_as_float(v0[j]), sl2, -m_use)) : 0.f;
-        const float a1 = ((mk.x >> (j + 1)) & 1u) ? fast_exp2(fmaf(__uint_as_float(v0[j + 1]), sl2, -m_use)) : 0.f;
-        const __nv_bfloat162 ba = __floats2bfloat162_rn(a0, a1);
-        l += a0 + a1;
-        lr += __low2float(ba) + __high2float(ba);
-        pk[j2] = *reinterpret_cast<const uint32_t*>(&ba);
-        const float b0 = ((mk.y >> j) & 1u) ? fast_exp2(fmaf(__uint_as_float(v1[j]), sl2, -m_use)) : 0.f;
-        const float b1 = ((mk.y >> (j + 1)) & 1u) ? fast_exp2(fmaf(__uint_as_float(v1[j + 1]), sl2, -m_use)) : 0.f;
-        const __nv_bfloat162 bb = __floats2bfloat162_rn(b0, b1);
-        l += b0 + b1;
-        lr += __low2float(bb) + __high2float(bb);
-        pk[16 + j2] = *reinterpret_cast<const uint32_t*>(&bb);
+      for (int j2 = 0; j2 < kCols / 2; ++j2) {
+        const float a0 = fast_exp2(fmaf(x[2 * j2], sl2, -m_use));
+        const float a1 = fast_exp2(fmaf(x[2 * j2 + 1], sl2, -m_use));
+        const uint32_t w = pack_bf16x2(a0, a1);
+        la[j2 & 3] += a0 + a1;
+        lra[j2 & 3] += __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
+        pk[j2] = w;
       }
-      tmem_st32(tmem + lane_base + kColP + 64 * s + 32 * sub, pk);
+      l += (la[0] + la[1]) + (la[2] + la[3]);
+      lr += (lra[0] + lra[1]) + (lra[2] + lra[3]);
+      static_assert(kCols == 64, "one 32-column TMEM store of P per softmax warp");
+      tmem_st32(tmem + lane_base + kColP + 64 * s + (kCols / 2) * sub, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[B_PFULL + s]);
-      mk = mk_next;
+#pragma unroll
+      for (int w = 0; w < kWords; ++w) mk[w] = mk_next[w];
     }
-    // row sums over the quadrant's two warps
+    // row sums over the quadrant's warps
     redl[(0 * kSubs + sub) * 128 + r] = l;
     redl[(1 * kSubs + sub) * 128 + r] = lr;
     __syncwarp();
@@ -388,32 +421,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (nkt > 0) {
       const float inv = (ok && lrt > 0.f) ? 1.f / lrt : 0.f;
       const float lse_nat = (ok && lt > 0.f) ? (m_ref + log2f(lt)) * 0.69314718055994531f : -INFINITY;
-      const uint32_t ocol = tmem + lane_base + kColO + 64 * sub;
-      uint32_t o0[32], o1[32];
-      tmem_ld32_sync(ocol, o0);
-      tmem_ld32_sync(ocol + 32, o1);
-      if (row_ok) {
-        uint4* dst = reinterpret_cast<uint4*>(p.out + (t * p.H + h) * kDvh + 64 * sub);
+      uint4* dst = reinterpret_cast<uint4*>(p.out + (t * p.H + h) * kDvh + kOCols * sub);
+#pragma unroll 1
+      for (int c = 0; c < kOCols / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32_sync(tmem + lane_base + kColO + kOCols * sub + 32 * c, o);
+        if (row_ok) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(o0[8 * j + 0]) * inv, __uint_as_float(o0[8 * j + 1]) * inv);
-          w.y = pack_bf16x2(__uint_as_float(o0[8 * j + 2]) * inv, __uint_as_float(o0[8 * j + 3]) * inv);
-          w.z = pack_bf16x2(__uint_as_float(o0[8 * j + 4]) * inv, __uint_as_float(o0[8 * j + 5]) * inv);
-          w.w = pack_bf16x2(__uint_as_float(o0[8 * j + 6]) * inv, __uint_as_float(o0[8 * j + 7]) * inv);
-          dst[j] = w;
+          for (int j = 0; j < 4; ++j) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(o[8 * j + 0]) * inv, __uint_as_float(o[8 * j + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(o[8 * j + 2]) * inv, __uint_as_float(o[8 * j + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(o[8 * j + 4]) * inv, __uint_as_float(o[8 * j + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(o[8 * j + 6]) * inv, __uint_as_float(o[8 * j + 7]) * inv);
+            dst[4 * c + j] = w;
+          }
         }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(o1[8 * j + 0]) * inv, __uint_as_float(o1[8 * j + 1]) * inv);
-          w.y = pack_bf16x2(__uint_as_float(o1[8 * j + 2]) * inv, __uint_as_float(o1[8 * j + 3]) * inv);
-          w.z = pack_bf16x2(__uint_as_float(o1[8 * j + 4]) * inv, __uint_as_float(o1[8 * j + 5]) * inv);
-          w.w = pack_bf16x2(__uint_as_float(o1[8 * j + 6]) * inv, __uint_as_float(o1[8 * j + 7]) * inv);
-          dst[4 + j] = w;
-        }
-        if (sub == 0 && p.lse) p.lse[t * p.H + h] = lse_nat;
       }
+      if (row_ok && sub == 0 && p.lse) p.lse[t * p.H + h] = lse_nat;
     }
   }
   tc_fence_before();
@@ -438,8 +463,11 @@ int launch_masked_mha(const BatchDev& b, const void* plan, const void* q, const 
   PlanView pv = plan_view(const_cast<void*>(plan), b.B, b.T);
   const int ldw = masked_mha_ldw(b.max_seq_len);
   uint32_t* mask = static_cast<uint32_t*>(ws);
-  cudaError_t ce = launch_pdl(mha_mask_kernel, dim3(b.T), dim3(256), sizeof(uint32_t) * ldw, stream,
-                              static_cast<const int32_t*>(pv.row_pos), S, topk, ldw, mask, &pv.hdr->status);
+  // rows per mask block: up to 8, within 48 KB of shared memory (ldw <= 2048 words)
+  const int mrows = std::max(1, std::min(8, 12288 / ldw));
+  cudaError_t ce = launch_pdl(mha_mask_kernel, dim3((b.T + mrows - 1) / mrows), dim3(32 * mrows),
+                              sizeof(uint32_t) * mrows * ldw, stream, static_cast<const int32_t*>(pv.row_pos), S,
+                              topk, ldw, b.T, mask, &pv.hdr->status);
   if (ce != cudaSuccess) return static_cast<int>(ce);
 
   MhaParams prm{};
