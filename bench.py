@@ -18,9 +18,10 @@ The JSON line also carries
                 queries and batch metadata go host->device and the output comes back; the paged
                 caches stay resident (they are the cache, not per-step inputs);
   cpu_baseline  the CPU oracle (float64 numpy) timed on this host on a bounded sample of rows;
-  short_prefill the masked MHA mode (the dense fallback for short prefill) on its own shape,
-                L = 2048, 16 heads, k = 512: mask + attention kernels, event-timed, in TFLOP/s
-                of the dense causal work against the measured bf16 peak.
+  short_prefill the masked MHA mode (the dense fallback for short prefill) on two shapes of its
+                own, L = 2048 with 16 heads and k = 512, and L = 4096 with 128 heads and k = 2048:
+                mask + attention kernels, event-timed, in TFLOP/s of the dense causal work
+                against the measured bf16 peak.
 `--impl reference` times that oracle alone as the reference arm.
 """
 from __future__ import annotations
@@ -189,15 +190,14 @@ class ClockSampler:
 # ---------------------------------------------------------------------------------------------
 # oracle timing (CPU baseline / reference arm)
 
-def short_prefill_mha(dev, timed_mean, n, tf_peak):
-    """The masked MHA mode (expanded heads, the DSA mask) on the short-prefill shape: one request
-    of 2048 positions, 16 heads, k = 512. The index sets are random valid sets (the dense tiles'
-    work does not depend on which positions are selected). Algorithmic work: the causal pairs
-    L(L+1)/2 times 2H(192 + 128) FLOPs."""
+def short_prefill_mha(dev, timed_mean, n, tf_peak, wl, label):
+    """The masked MHA mode (expanded heads, the DSA mask) on one whole-prefill request of workload
+    `wl` (its length, heads and k). The index sets are random valid sets (the dense tiles' work does
+    not depend on which positions are selected). Algorithmic work: the causal pairs L(L+1)/2 times
+    2H(192 + 128) FLOPs."""
     import torch
     import sparse_attention_12_b200 as dsa
     from sparse_attention_12_b200 import synth
-    wl = synth.workload("prefill_2048")
     L, H, k = int(wl.seq_lens[0]), wl.n_heads, wl.topk
     x = synth.make_mha_inputs(wl, seed=0)
     S = torch.from_numpy(synth.random_index_sets(wl.seq_lens, wl.q_per_req, k, seed=0)).to(dev)
@@ -220,7 +220,7 @@ def short_prefill_mha(dev, timed_mean, n, tf_peak):
     ms = timed_mean(fn, n)
     flops = L * (L + 1) / 2 * 2 * H * (192 + 128)
     tf = flops / (ms / 1e3) / 1e12
-    return {"workload": "prefill_2048 (masked MHA mode)", "us": 1e3 * ms, "algorithmic_flops": flops,
+    return {"workload": label, "us": 1e3 * ms, "algorithmic_flops": flops,
             "TFLOPs": tf, "peak_TFLOPs": tf_peak, "frac": tf / tf_peak, "launches": 2,
             "note": "mask kernel + attention kernel, one call, event-timed; random valid index sets"}
 
@@ -433,7 +433,12 @@ def main():
 
     short = None
     if not args.no_short_prefill:
-        short = short_prefill_mha(dev, timed_mean, max(3, min(args.steps, 20)), tf_peak)
+        reps = max(3, min(args.steps, 20))
+        short = [short_prefill_mha(dev, timed_mean, reps, tf_peak, synth.workload("prefill_2048"),
+                                   "prefill_2048 (masked MHA mode): L 2048, 16 heads, k 512"),
+                 short_prefill_mha(dev, timed_mean, reps, tf_peak,
+                                   synth.custom("prefill_4k_128h", [4096], [4096], n_heads=128, topk=2048),
+                                   "masked MHA mode at the model's head count: L 4096, 128 heads, k 2048")]
 
     # end to end through the public API with host buffers
     e2e = None

@@ -90,6 +90,11 @@ def test_masked_mha_prefill_2048_shape():
     _run([2048], H=16, topk=512, seed=4, rows=rows)
 
 
+def test_masked_mha_128_heads():
+    """The model's head count (128 CTAs per query tile along the head axis), two requests, all rows."""
+    _run([300, 77], H=128, topk=128, seed=6)
+
+
 def test_masked_mha_rejects_requests_with_a_cached_prefix():
     """n_b != m_b is not a whole prefill: the kernel records DSA_ERR_DEVICE_INDEX and writes nothing."""
     lens, qs = [200], [100]
