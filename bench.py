@@ -491,6 +491,14 @@ def main():
         cpu = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                "sample": f"{rows} of the {T} query rows of {wl.name} through the whole path in "
                          f"{dt:.1f} s (float64 numpy, BLAS threads)"}
+        try:  # the same oracle on one thread, a smaller sample
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1):
+                r1, n1, d1 = time_oracle(hb, budget_s=4.0)
+            cpu["single_thread"] = {"value": r1, "unit": UNIT, "cores": 1,
+                                    "sample": f"{n1} query rows in {d1:.1f} s"}
+        except ImportError:
+            pass
 
     launches_per_step = 3 + (1 if mla_ws_n > 0 else 0) + (1 if topk_ws_n > 0 else 0)
     line = {
