@@ -3,32 +3,37 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
 One step = the three kernels of one layer -- Lightning-Indexer scores, top-k, sparse MLA -- over one
-batch of the workload through the C ABI (dsa_index_scores, dsa_topk, dsa_sparse_mla), inputs resident
+batch of a workload through the C ABI (dsa_index_scores, dsa_topk, dsa_sparse_mla), inputs resident
 in HBM, with the batch plan computed once per batch (it depends only on the batch's lengths, so a
-model computes it once per forward pass for all its layers). `layer_with_plan_us` is the whole
-`dsa_layer` call, plan included, and `plan_us` the plan alone. Each timed step is bracketed by CUDA
-events on the launching stream, with a 256 MiB L2 flush (untimed) between steps. Under torchrun every rank runs
-its own batch (weak scaling, no collective on the data path); rank 0 prints one JSON line with the
-max-over-ranks time.
+model computes it once per forward pass for all its layers). Each timed step is bracketed by CUDA
+events on the launching stream, with a 256 MiB L2 flush (untimed) between steps.
 
-The JSON line also carries
-  roofline      the dominant kernel's achieved algorithmic bytes/s against the measured HBM peak,
-                from per-stage CUDA-event timings of the same kernels;
-  e2e           the same metric through the public API with host (pinned) inputs: per step the
-                queries and batch metadata go host->device and the output comes back; the paged
-                caches stay resident (they are the cache, not per-step inputs);
+The headline (`value`, `ms_per_step`, `config`) is prefill_32k, the workload with the most work that
+one GPU holds (1 sequence of 32768 positions, 64 indexer heads, k = 2048, 128 MLA heads). At
+--gpus 1 the line also carries a `workloads` block that measures all five workload shapes the same
+way: layer µs, query tok/s, and per stage its µs, its algorithmic bytes and FLOPs, the bound that
+applies to it (HBM, FP8 tensor or bf16 tensor, whichever roofline time is longer) and its fraction
+of that roofline; for the decode shapes also the top-k + sparse-MLA gather fraction of HBM.
+
+Other keys of the JSON line:
+  roofline      the headline's dominant kernel against the bound that applies to it;
+  peaks         the denominators: HBM and bf16 from MEASURED_PEAKS.json, FP8 measured in this
+                process (torch._scaled_mm e4m3, 8192^3, best of 10);
+  e2e           the headline through the public API (dsa_layer) with host (pinned) inputs: per
+                step the queries and batch metadata go host->device and the output comes back;
+                the paged caches stay resident (they are the cache, not per-step inputs). Copies
+                of step i+1 overlap the layer of step i on separate streams;
   cpu_baseline  the CPU oracle (float64 numpy) timed on this host on a bounded sample of rows;
-  short_prefill the masked MHA mode (the dense fallback for short prefill) on two shapes of its
-                own, L = 2048 with 16 heads and k = 512, and L = 4096 with 128 heads and k = 2048:
-                mask + attention kernels, event-timed, in TFLOP/s of the dense causal work
-                against the measured bf16 peak.
-`--impl reference` times that oracle alone as the reference arm.
+  short_prefill the masked MHA mode (the dense fallback for short prefill) on two shapes.
+Under torchrun every rank runs its own batch of the headline workload (weak scaling, no collective
+on the data path); rank 0 prints one JSON line with the max-over-ranks time.
+`--impl reference` times the oracle alone as the reference arm: each step a bounded random sample
+of the headline workload's query rows, each row through the whole path.
 """
 from __future__ import annotations
 
 import argparse
 import json
-import math
 import os
 import statistics
 import sys
@@ -42,8 +47,11 @@ sys.path.insert(0, ROOT)
 
 METRIC = "DSA layer µs (indexer+top-k+sparse MLA), query tok/s; % of HBM/FP8 roofline"
 UNIT = "query tok/s"
-DEFAULT_WORKLOAD = "decode_64x16k"
+HEADLINE = "prefill_32k"
+ALL_WORKLOADS = ("prefill_2048", "decode_64x16k", "mtp_16x128k", "prefill_32k", "mixed_128")
+DECODE_WORKLOADS = ("decode_64x16k", "mtp_16x128k", "mixed_128")
 L2_FLUSH_BYTES = 256 << 20
+REF_ROWS_PER_STEP = 32
 
 
 def recorded_traffic(kernel: str, workload: str):
@@ -54,7 +62,8 @@ def recorded_traffic(kernel: str, workload: str):
     try:
         with open(path) as f:
             rec = json.load(f)[kernel]
-        if rec["workload"] != workload:
+        rec = rec[workload] if workload in rec else rec
+        if rec.get("workload") != workload:
             return None
         with open(os.path.join(ROOT, rec["source"]), "rb") as f:
             if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
@@ -64,14 +73,43 @@ def recorded_traffic(kernel: str, workload: str):
         return None
 
 
-def measured_peaks():
+def file_peaks():
+    """HBM GB/s and bf16 TFLOP/s (burst, sustained) from MEASURED_PEAKS.json, else the fallback."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+        return {"hbm_GBps": float(d["hbm_gbs"]), "bf16_TFLOPs": float(d["bf16_tflops"]),
+                "bf16_TFLOPs_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured (MEASURED_PEAKS.json)"}
     except Exception:
-        return 6650.0, 1590.0, "fallback"
+        return {"hbm_GBps": 6650.0, "bf16_TFLOPs": 1590.0, "bf16_TFLOPs_sustained": 1400.0, "source": "fallback"}
+
+
+def measure_fp8_peak(dev, n: int = 8192, reps: int = 10):
+    """Dense FP8 (e4m3 x e4m3 -> bf16, fp32 accumulate) GEMM throughput of cuBLAS through
+    torch._scaled_mm, n^3, best of `reps` CUDA-event timings. None if unavailable."""
+    import torch
+    try:
+        g = torch.Generator(device=dev).manual_seed(1)
+        a = torch.randn((n, n), device=dev, generator=g).to(torch.float8_e4m3fn)
+        b = torch.randn((n, n), device=dev, generator=g).to(torch.float8_e4m3fn)
+        one = torch.ones((), device=dev, dtype=torch.float32)
+        f = lambda: torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        for _ in range(3):
+            f()
+        best = float("inf")
+        for _ in range(reps):
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            f()
+            e.record()
+            e.synchronize()
+            best = min(best, s.elapsed_time(e))
+        del a, b
+        return 2.0 * n ** 3 / (best / 1e3) / 1e12
+    except Exception:
+        return None
 
 
 # ---------------------------------------------------------------------------------------------
@@ -79,7 +117,7 @@ def measured_peaks():
 
 def algorithmic(hb):
     """Bytes each kernel must move and FLOPs it must do for one step of this batch."""
-    req, pos = _positions(hb)
+    req, pos = hb.row_positions()
     T = hb.total_q
     nhI = hb.qI.shape[1]
     H = hb.q.shape[1]
@@ -96,14 +134,48 @@ def algorithmic(hb):
     idx_bytes = int(keys_per_req.sum()) * (128 + 4) + T * (nhI * 128 + 4 + nhI * 4) + int(vis.sum()) * 4
     idx_flops = int(vis.sum()) * 2 * nhI * 128
     topk_bytes = int(vis.sum()) * 4 + T * k * 4
-    mla_bytes = int(sel.sum()) * (576 * 2 + 4) + T * H * 576 * 2 + T * H * 512 * 2
+    # sparse MLA: every latent row a request's index sets name, once (at most the request's whole
+    # cache: a long prefill's rows are read from HBM once and re-read from L2), the indices, the
+    # queries and the output
+    rows_per_req = 0
+    for b in range(len(hb.seq_lens)):
+        lo, hi = int(hb.cu_q[b]), int(hb.cu_q[b + 1])
+        if hi > lo:
+            rows_per_req += min(int(hb.seq_lens[b]), int(sel[lo:hi].sum()))
+    mla_bytes = rows_per_req * 576 * 2 + int(sel.sum()) * 4 + T * H * 576 * 2 + T * H * 512 * 2
     mla_flops = int(sel.sum()) * (2 * H * 576 + 2 * H * 512)
     return dict(index_scores=(idx_bytes, idx_flops), topk=(topk_bytes, 0), sparse_mla=(mla_bytes, mla_flops))
 
 
-def _positions(hb):
-    req, pos = hb.row_positions()
-    return req, pos
+# the tensor dtype of each stage's contraction (the indexer is FP8, the sparse MLA bf16)
+STAGE_TENSOR = {"index_scores": "fp8", "topk": None, "sparse_mla": "bf16"}
+
+
+def stage_roofline(name: str, nbytes: int, flops: int, us: float, peaks: dict) -> dict:
+    """A stage against the bound that applies to it: the longer of its HBM time (algorithmic bytes
+    over the measured copy bandwidth) and its tensor time (FLOPs over the measured peak of its own
+    dtype). `frac` = roofline time / measured time = achieved / peak in the bound's unit."""
+    t_hbm = nbytes / (peaks["hbm_GBps"] * 1e9)
+    kind = STAGE_TENSOR[name]
+    tf_peak = None
+    if kind == "fp8":
+        tf_peak = peaks["fp8_TFLOPs"]
+    elif kind == "bf16":
+        tf_peak = peaks["bf16_TFLOPs"]
+    t_tc = flops / (tf_peak * 1e12) if (tf_peak and flops) else 0.0
+    s = us / 1e6
+    r = {"us": us, "algorithmic_bytes": int(nbytes), "algorithmic_flops": int(flops),
+         "GBps": nbytes / s / 1e9, "TFLOPs": flops / s / 1e12 if flops else 0.0}
+    if t_tc > t_hbm:
+        r.update(bound="tensor", unit="TFLOP/s", achieved=flops / s / 1e12, peak=tf_peak, dtype=kind,
+                 roofline_us=1e6 * t_tc, frac=t_tc / s)
+    else:
+        r.update(bound="hbm", unit="GB/s", achieved=nbytes / s / 1e9, peak=peaks["hbm_GBps"],
+                 roofline_us=1e6 * t_hbm, frac=t_hbm / s)
+    if kind:  # the other fraction too, for the stages that have both
+        r["hbm_frac"] = t_hbm / s
+        r["tensor_frac"] = t_tc / s if tf_peak else None
+    return r
 
 
 # ---------------------------------------------------------------------------------------------
@@ -129,12 +201,20 @@ def job_throughput(rows_per_rank: int, world: int, ms: float) -> float:
     return world * rows_per_rank / (ms / 1e3)
 
 
+def config_of(wl, world: int) -> dict:
+    """The `config` object of the JSON line (the same for both arms)."""
+    return {"workload": wl.name, "requests": wl.batch, "query_rows": wl.total_q, "context": max(wl.seq_lens),
+            "topk": wl.topk, "index_heads": wl.n_heads_index, "heads": wl.n_heads, "page_size": 64,
+            "l2": "256 MiB flush between timed steps", "parallelism": f"{world} independent ranks",
+            "step": "dsa_index_scores + dsa_topk + dsa_sparse_mla, batch plan computed once per batch"}
+
+
 # ---------------------------------------------------------------------------------------------
-# clocks sampled during the timed region
+# clocks sampled during the timed regions
 
 class ClockSampler:
-    """Samples SM clock and clock-event reasons every few ms while the timed region runs (NVML reads
-    only; nothing is set). Falls back to nvidia-smi's loop mode when NVML is unavailable."""
+    """Samples SM clock and clock-event reasons every few ms while a timed region runs (NVML reads
+    only; nothing is set). Use as a context manager around each timed region; samples accumulate."""
 
     # NVML clocks-event reason bits
     REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
@@ -145,11 +225,22 @@ class ClockSampler:
         self.period = period_s
         self.samples = []
         self.max_mhz = None
-        self._stop = threading.Event()
+        self._nvml = None
+        self._h = None
+        self._stop = None
         self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._nvml = pynvml
+        except Exception:
+            self._nvml = None
 
-    def _run(self, pynvml, h):
-        while not self._stop.is_set():
+    def _run(self, stop):
+        pynvml, h = self._nvml, self._h
+        while not stop.is_set():
             try:
                 mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
                 try:
@@ -162,21 +253,17 @@ class ClockSampler:
             time.sleep(self.period)
 
     def __enter__(self):
-        try:
-            import pynvml
-            pynvml.nvmlInit()
-            h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
-            self._thread = threading.Thread(target=self._run, args=(pynvml, h), daemon=True)
+        if self._nvml is not None:
+            self._stop = threading.Event()
+            self._thread = threading.Thread(target=self._run, args=(self._stop,), daemon=True)
             self._thread.start()
-        except Exception:
-            self._thread = None
         return self
 
     def __exit__(self, *exc):
-        self._stop.set()
         if self._thread is not None:
+            self._stop.set()
             self._thread.join(timeout=2)
+            self._thread = None
 
     def summary(self):
         if not self.samples:
@@ -190,14 +277,241 @@ class ClockSampler:
 # ---------------------------------------------------------------------------------------------
 # oracle timing (CPU baseline / reference arm)
 
-def short_prefill_mha(dev, timed_mean, n, tf_peak, wl, label):
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n and n[0]:
+            return int(n[0])
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_rows(hb, rows):
+    """The whole path (scores over the visible prefix, full-sort TopK, attention on S_t) of the
+    oracle for the given query rows; returns the seconds it took."""
+    from oracle import dsa_oracle as O
+    req, pos = O.query_positions(hb.seq_lens, hb.cu_q)
+    t0 = time.perf_counter()
+    for t in rows:
+        I = O.index_scores_row(int(t), req, pos, hb.block_table, hb.qI, hb.qI_scale, hb.wI, hb.kI_cache,
+                               hb.kI_scale)
+        S = O.topk_select(I, hb.wl.topk)
+        O.sparse_mla_row(int(t), req, S, hb.block_table, hb.q, hb.kv_cache, hb.wl.softmax_scale)
+    return time.perf_counter() - t0
+
+
+def time_oracle(hb, budget_s: float = 12.0, seed: int = 0):
+    """The oracle on uniformly drawn query rows until `budget_s` passes; returns (rows/s, rows,
+    seconds). Rows drawn uniformly make rows/s an unbiased estimate for the whole step."""
+    T = hb.total_q
+    order = np.random.default_rng(seed).permutation(T)
+    done, secs = 0, 0.0
+    for t in order:
+        secs += oracle_rows(hb, [t])
+        done += 1
+        if secs > budget_s:
+            break
+    return done / secs, done, secs
+
+
+def reference_arm(args, wl, world):
+    """The oracle as the reference arm: each step is REF_ROWS_PER_STEP uniformly drawn query rows
+    of the workload (a new draw every step), each through the whole path; ms_per_step is the
+    measured time of that sample, value its rows per second."""
+    from sparse_attention_12_b200 import synth
+    hb = synth.make_batch(wl, seed=0)
+    rng = np.random.default_rng(1)
+    T = hb.total_q
+    R = min(REF_ROWS_PER_STEP, T)
+    for _ in range(args.warmup):
+        oracle_rows(hb, rng.choice(T, size=1))
+    secs = [oracle_rows(hb, rng.choice(T, size=R, replace=False)) for _ in range(args.steps)]
+    s = statistics.mean(secs)
+    value = R / s
+    cores = blas_threads()
+    sample = (f"{R} uniformly drawn query rows of {wl.name} per step ({args.steps} steps, a new draw each), "
+              f"each through the whole path (float64 numpy: scores over the visible prefix, full sort, "
+              f"attention on S_t); value = rows per second of the measured steps")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * s, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(wl, world), "rows_per_step": R,
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------------------------------------
+# one workload on the GPU
+
+class Runner:
+    """Device copies of one workload's batch and the three stage calls of a step."""
+
+    def __init__(self, dsa, torch, hb, dev):
+        self.hb, self.dev = hb, dev
+        self.db = db = dsa.DeviceBatch(hb, device=dev)
+        T = hb.total_q
+        self.T = T
+        self.out = torch.empty((T, db.H, 512), dtype=torch.bfloat16, device=dev)
+        self.ws = torch.empty(max(16, dsa.layer_workspace_size(db.batch, db.nhI, db.H, db.k)), dtype=torch.uint8,
+                              device=dev)
+        self.plan = dsa.plan(db.batch, db.nhI)
+        ld = (hb.max_seq_len + 127) // 128 * 128
+        self.scores = torch.empty((T, ld), dtype=torch.float32, device=dev)
+        self.S = torch.empty((T, db.k), dtype=torch.int32, device=dev)
+        lib = dsa.load()
+        self.mla_ws_n = lib.dsa_sparse_mla_workspace_size(db.batch.ref(), db.H, db.k)
+        mla_ws = torch.empty(max(16, self.mla_ws_n), dtype=torch.uint8, device=dev)
+        self.topk_ws_n = lib.dsa_topk_workspace_size(db.batch.ref(), db.k)
+        topk_ws = torch.empty(max(16, self.topk_ws_n), dtype=torch.uint8, device=dev) if self.topk_ws_n else None
+        self.stages = {
+            "index_scores": lambda: dsa.index_scores(db.batch, self.plan, db.qI, db.qI_scale, db.wI, db.kI_cache,
+                                                     db.kI_scale, scores=self.scores, ld=ld),
+            "topk": lambda: dsa.topk(db.batch, self.plan, self.scores, db.k, S=self.S, ws=topk_ws),
+            "sparse_mla": lambda: dsa.sparse_mla(db.batch, self.plan, db.q, db.kv_cache, self.S, db.softmax_scale,
+                                                 out=self.out, ws=mla_ws),
+        }
+        self.layer = lambda: dsa.layer(db.batch, db.qI, db.qI_scale, db.wI, db.kI_cache, db.kI_scale, db.q,
+                                       db.kv_cache, db.k, db.softmax_scale, out=self.out, ws=self.ws)
+        self.replan = lambda: dsa.plan(db.batch, db.nhI, self.plan)
+
+    def step(self):
+        for fn in self.stages.values():
+            fn()
+
+    def launches_per_step(self):
+        """Kernels of the library one step launches: the three stages, plus the top-k merge for rows
+        longer than one slice and the split combine when index sets are split across clusters."""
+        return 3 + (1 if self.mla_ws_n > 0 else 0) + (1 if self.topk_ws_n > 0 else 0)
+
+
+def timed_steps(torch, fn, n, flush, stream):
+    """Mean ms of `fn` over n runs, each bracketed by CUDA events on `stream`, L2 flushed before."""
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for i in range(n):
+        flush.fill_(i & 0xFF)
+        starts[i].record(stream)
+        fn()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    return statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
+
+
+def measure_workload(dsa, torch, wl, dev, seed, steps, warmup, flush, sampler, peaks, dist=None):
+    """Layer time (the three stages back to back), the dsa_layer call, and per-stage times, each
+    event-timed with an L2 flush before every run; returns (report, runner)."""
+    from sparse_attention_12_b200 import synth
+    hb = synth.make_batch(wl, seed=seed)
+    r = Runner(dsa, torch, hb, dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(warmup, 0)):
+        r.step()
+        r.layer()
+    torch.cuda.synchronize()
+    for plan_ws in (r.plan, r.ws):  # the layer call keeps its plan at the start of its workspace
+        status = dsa.status_read(plan_ws)
+        if status != 0:
+            raise RuntimeError(f"{wl.name}: device status {status} after warm-up")
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        ms = timed_steps(torch, r.step, steps, flush, stream)
+    ms = max_over_ranks(ms, dist, dev)
+    n_extra = max(3, min(steps, 10))
+    layer_ms = max_over_ranks(timed_steps(torch, r.layer, n_extra, flush, stream), dist, dev)
+    plan_ms = max_over_ranks(timed_steps(torch, r.replan, n_extra, flush, stream), dist, dev)
+    stage_ms = {n: timed_steps(torch, fn, n_extra, flush, stream) for n, fn in r.stages.items()}
+    work = algorithmic(hb)
+    stages = {n: stage_roofline(n, work[n][0], work[n][1], 1e3 * stage_ms[n], peaks) for n in r.stages}
+    layer_roof_us = sum(s["roofline_us"] for s in stages.values())
+    rep = {"workload": wl.name, "query_rows": hb.total_q, "steps": steps, "layer_us": 1e3 * ms,
+           "q_tok_s": hb.total_q / (ms / 1e3), "layer_with_plan_us": 1e3 * layer_ms, "plan_us": 1e3 * plan_ms,
+           "layer_roofline_us": layer_roof_us, "layer_frac": layer_roof_us / (1e3 * ms),
+           "launches_per_step": r.launches_per_step(), "stages": stages}
+    if wl.name in DECODE_WORKLOADS or hb.total_q <= 256:
+        # the north star's composite: the top-k and the gather/attention together against HBM
+        tb = stages["topk"]["algorithmic_bytes"] + stages["sparse_mla"]["algorithmic_bytes"]
+        tu = stages["topk"]["us"] + stages["sparse_mla"]["us"]
+        rep["topk_plus_gather"] = {"algorithmic_bytes": tb, "us": tu, "GBps": tb / (tu / 1e6) / 1e9,
+                                   "frac": tb / (tu / 1e6) / 1e9 / peaks["hbm_GBps"]}
+    return rep, r
+
+
+def e2e_pipelined(dsa, torch, r, hb, dev, steps, warmup, dist=None):
+    """The headline through dsa_layer with host inputs: every step copies its inputs host->device from
+    pinned memory and its output device->host. Copies run on their own streams, double-buffered, so
+    step i+1's upload and step i-1's download overlap step i's layer; ms = the whole run / steps."""
+    db = r.db
+    T = hb.total_q
+    pin = lambda t: t.cpu().pin_memory()
+    h_in = {"qI": pin(db.qI.view(torch.uint8)), "qI_scale": pin(db.qI_scale), "wI": pin(db.wI), "q": pin(db.q),
+            "seq_lens": pin(db.batch.seq_lens), "cu_q": pin(db.batch.cu_q), "block_table": pin(db.batch.block_table)}
+    d_in = [{n: torch.empty_like(t, device=dev) for n, t in h_in.items()} for _ in range(2)]
+    outs = [torch.empty_like(r.out) for _ in range(2)]
+    wss = [r.ws, torch.empty_like(r.ws)]
+    h_out = [torch.empty(r.out.shape, dtype=r.out.dtype).pin_memory() for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+    d2h = h_out[0].numel() * h_out[0].element_size()
+    batches = [dsa.Batch(d["seq_lens"], d["cu_q"], d["block_table"], hb.num_pages, T, db.batch.c.max_q,
+                         hb.max_seq_len) for d in d_in]
+    s_up, s_comp, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+
+    def run(n):
+        up_done = [None, None]
+        comp_done = [None, None]
+        down_done = [None, None]
+        for i in range(n):
+            b = i & 1
+            with torch.cuda.stream(s_up):
+                if comp_done[b] is not None:
+                    s_up.wait_event(comp_done[b])  # buffer set b is free once step i-2's layer ran
+                for k in h_in:
+                    d_in[b][k].copy_(h_in[k], non_blocking=True)
+                up_done[b] = ev()
+                up_done[b].record(s_up)
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(up_done[b])
+                if down_done[b] is not None:
+                    s_comp.wait_event(down_done[b])  # output b was read back (step i-2)
+                dsa.layer(batches[b], d_in[b]["qI"].view(torch.float8_e4m3fn), d_in[b]["qI_scale"], d_in[b]["wI"],
+                          db.kI_cache, db.kI_scale, d_in[b]["q"], db.kv_cache, db.k, db.softmax_scale, out=outs[b],
+                          ws=wss[b])
+                comp_done[b] = ev()
+                comp_done[b].record(s_comp)
+            with torch.cuda.stream(s_down):
+                s_down.wait_event(comp_done[b])
+                h_out[b].copy_(outs[b], non_blocking=True)
+                down_done[b] = ev()
+                down_done[b].record(s_down)
+
+    run(max(warmup, 2))
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(s_up)
+    run(steps)
+    s_up.wait_stream(s_down)
+    z.record(s_up)
+    torch.cuda.synchronize()
+    e_ms = max_over_ranks(a.elapsed_time(z) / steps, dist, dev)
+    for d in d_in:
+        d.clear()
+    return {"value": None, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": e_ms, "steps": steps,
+            "note": "dsa_layer per step with its inputs copied from pinned host memory and its output copied "
+                    "back; uploads, layers and downloads on three streams, double-buffered"}
+
+
+def short_prefill_mha(dsa, torch, synth, dev, flush, n, tf_peak, wl, label):
     """The masked MHA mode (expanded heads, the DSA mask) on one whole-prefill request of workload
     `wl` (its length, heads and k). The index sets are random valid sets (the dense tiles' work does
     not depend on which positions are selected). Algorithmic work: the causal pairs L(L+1)/2 times
     2H(192 + 128) FLOPs."""
-    import torch
-    import sparse_attention_12_b200 as dsa
-    from sparse_attention_12_b200 import synth
     L, H, k = int(wl.seq_lens[0]), wl.n_heads, wl.topk
     x = synth.make_mha_inputs(wl, seed=0)
     S = torch.from_numpy(synth.random_index_sets(wl.seq_lens, wl.q_per_req, k, seed=0)).to(dev)
@@ -217,7 +531,7 @@ def short_prefill_mha(dev, timed_mean, n, tf_peak, wl, label):
     status = dsa.status_read(plan)
     if status != 0:
         raise RuntimeError(f"device status {status} in the masked MHA mode")
-    ms = timed_mean(fn, n)
+    ms = timed_steps(torch, fn, n, flush, torch.cuda.current_stream())
     flops = L * (L + 1) / 2 * 2 * H * (192 + 128)
     tf = flops / (ms / 1e3) / 1e12
     return {"workload": label, "us": 1e3 * ms, "algorithmic_flops": flops,
@@ -225,51 +539,22 @@ def short_prefill_mha(dev, timed_mean, n, tf_peak, wl, label):
             "note": "mask kernel + attention kernel, one call, event-timed; random valid index sets"}
 
 
-def blas_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
-        if n and n[0]:
-            return int(n[0])
-    except Exception:
-        pass
-    return os.cpu_count() or 1
-
-
-def time_oracle(hb, budget_s: float = 12.0, max_rows: int = 64):
-    """Run the oracle on a bounded sample of query rows; returns (rows/s, rows, seconds)."""
-    from oracle import dsa_oracle as O
-    req, pos = O.query_positions(hb.seq_lens, hb.cu_q)
-    T = hb.total_q
-    tau = hb.wl.softmax_scale
-    k = hb.wl.topk
-    order = np.random.default_rng(0).permutation(T)
-    done, t0 = 0, time.perf_counter()
-    for t in order[:max_rows]:
-        I = O.index_scores_row(int(t), req, pos, hb.block_table, hb.qI, hb.qI_scale, hb.wI, hb.kI_cache,
-                               hb.kI_scale)
-        S = O.topk_select(I, k)
-        O.sparse_mla_row(int(t), req, S, hb.block_table, hb.q, hb.kv_cache, tau)
-        done += 1
-        if time.perf_counter() - t0 > budget_s:
-            break
-    dt = time.perf_counter() - t0
-    return done / dt, done, dt
-
-
 # ---------------------------------------------------------------------------------------------
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=HEADLINE, help="headline workload")
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--only-headline", action="store_true", help="skip the block of the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-short-prefill", action="store_true")
     args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps")
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -281,31 +566,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return 0
-        hb = synth.make_batch(wl, seed=0)
-        budget = max(2.0, min(60.0, 8.0 * max(args.steps, 1) / max(args.steps + args.warmup, 1)))
-        for _ in range(args.warmup):
-            time_oracle(hb, budget_s=0.5, max_rows=1)
-        per_step = []
-        rows_total, secs_total = 0, 0.0
-        for _ in range(args.steps):
-            rate, rows, dt = time_oracle(hb, budget_s=budget / max(args.steps, 1), max_rows=hb.total_q)
-            per_step.append(hb.total_q / rate)   # seconds a full step would take at this rate
-            rows_total += rows
-            secs_total += dt
-        value = rows_total / secs_total
-        ms = 1e3 * hb.total_q / value
-        cores = blas_threads()
-        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": wl.name, "requests": wl.batch, "query_rows": wl.total_q,
-                           "context": max(wl.seq_lens), "topk": wl.topk, "index_heads": wl.n_heads_index,
-                           "heads": wl.n_heads},
-                "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                                 "sample": f"{rows_total} query rows of {wl.name}, full path per row, "
-                                           f"extrapolated to the {hb.total_q}-row step"},
-                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-        print(json.dumps(line), flush=True)
+        print(json.dumps(reference_arm(args, wl, world)), flush=True)
         return 0
 
     import torch
@@ -313,171 +574,37 @@ def main():
 
     dist = None
     if world > 1:
-        import torch.distributed as dist
         import datetime
+        import torch.distributed as dist
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local_rank if world > 1 else 0)
     torch.cuda.set_device(dev)
     dsa.load()
 
-    hb = synth.make_batch(wl, seed=rank_seed(rank))
-    db = dsa.DeviceBatch(hb, device=dev)
-    T = hb.total_q
-    stream = torch.cuda.current_stream()
-    out = torch.empty((T, db.H, 512), dtype=torch.bfloat16, device=dev)
-    ws = torch.empty(max(16, dsa.layer_workspace_size(db.batch, db.nhI, db.H, db.k)), dtype=torch.uint8, device=dev)
+    peaks = file_peaks()
+    fp8 = measure_fp8_peak(dev)
+    peaks["fp8_TFLOPs_nominal_ratio"] = 2.0 * peaks["bf16_TFLOPs"]
+    peaks["fp8_TFLOPs"] = fp8 if fp8 else peaks["fp8_TFLOPs_nominal_ratio"]
+    peaks["fp8_source"] = ("measured in this process: torch._scaled_mm e4m3 x e4m3 -> bf16, 8192^3, best of 10"
+                           if fp8 else "2 x the bf16 peak (nominal FP8/bf16 ratio)")
+
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-
-    # the batch plan, once per batch; the layer's three kernels per step
-    plan_t = dsa.plan(db.batch, db.nhI)
-    ld = (hb.max_seq_len + 127) // 128 * 128
-    scores = torch.empty((T, ld), dtype=torch.float32, device=dev)
-    S = torch.empty((T, db.k), dtype=torch.int32, device=dev)
-    mla_ws_n = dsa.load().dsa_sparse_mla_workspace_size(db.batch.ref(), db.H, db.k)
-    mla_ws = torch.empty(max(16, mla_ws_n), dtype=torch.uint8, device=dev)
-    topk_ws_n = dsa.load().dsa_topk_workspace_size(db.batch.ref(), db.k)
-    topk_ws = torch.empty(max(16, topk_ws_n), dtype=torch.uint8, device=dev) if topk_ws_n else None
-    stages = {
-        "index_scores": lambda: dsa.index_scores(db.batch, plan_t, db.qI, db.qI_scale, db.wI, db.kI_cache,
-                                                 db.kI_scale, scores=scores, ld=ld),
-        "topk": lambda: dsa.topk(db.batch, plan_t, scores, db.k, S=S, ws=topk_ws),
-        "sparse_mla": lambda: dsa.sparse_mla(db.batch, plan_t, db.q, db.kv_cache, S, db.softmax_scale, out=out,
-                                             ws=mla_ws),
-    }
-
-    def step():
-        for fn in stages.values():
-            fn()
-
-    def layer_call():
-        dsa.layer(db.batch, db.qI, db.qI_scale, db.wI, db.kI_cache, db.kI_scale, db.q, db.kv_cache, db.k,
-                  db.softmax_scale, out=out, ws=ws)
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    for _ in range(max(args.warmup, 0)):
-        step()
-        layer_call()
-    torch.cuda.synchronize()
-    for plan_ws in (plan_t, ws):  # the layer call keeps its plan at the start of its workspace
-        status = dsa.status_read(plan_ws)
-        if status != 0:
-            raise RuntimeError(f"device status {status} after warm-up")
-
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     sampler = ClockSampler(dev.index if dev.index is not None else 0)
-    barrier()
-    with sampler:
-        for i in range(args.steps):
-            flush.fill_(i & 0xFF)
-            starts[i].record(stream)
-            step()
-            ends[i].record(stream)
-        barrier()
-    times = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    ms = max_over_ranks(statistics.mean(times), dist, dev)
+
+    head, r = measure_workload(dsa, torch, wl, dev, rank_seed(rank), args.steps, args.warmup, flush, sampler,
+                               peaks, dist)
+    ms = head["layer_us"] / 1e3
+    T = head["query_rows"]
     value = job_throughput(T, world, ms)
 
-    # the whole dsa_layer call (plan included) and the plan alone, same protocol
-    def timed_mean(fn, n):
-        ts = []
-        for i in range(n):
-            flush.fill_(i & 0xFF)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            fn()
-            b.record(stream)
-            b.synchronize()
-            ts.append(a.elapsed_time(b))
-        return statistics.mean(ts)
-
-    n_extra = max(3, min(args.steps, 50))
-    layer_plan_ms = max_over_ranks(timed_mean(layer_call, n_extra), dist, dev)
-    plan_ms = max_over_ranks(timed_mean(lambda: dsa.plan(db.batch, db.nhI, plan_t), n_extra), dist, dev)
-
-    # per-stage timings of the same kernels (roofline of the dominant one)
-    stage_ms = {n: [] for n in stages}
-    for i in range(max(3, min(args.steps, 20))):
-        for name, fn in stages.items():
-            flush.fill_(i & 0xFF)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            fn()
-            b.record(stream)
-            b.synchronize()
-            stage_ms[name].append(a.elapsed_time(b))
-    stage_ms = {n: statistics.mean(v) for n, v in stage_ms.items()}
-    work = algorithmic(hb)
-    hbm_peak, tf_peak, peak_src = measured_peaks()
-    dominant = max(stage_ms, key=stage_ms.get)
-    dom_bytes = work[dominant][0]
-    achieved = dom_bytes / (stage_ms[dominant] / 1e3) / 1e9
-    stage_report = {n: {"us": 1e3 * stage_ms[n], "GBps": work[n][0] / (stage_ms[n] / 1e3) / 1e9,
-                        "TFLOPs": work[n][1] / (stage_ms[n] / 1e3) / 1e12 if work[n][1] else 0.0}
-                    for n in stages}
-    total_bytes = sum(w[0] for w in work.values())
-
-    # the step before the layer: writing every query row's new key and latent row into the caches
-    # (not part of the step; timed after the layer measurements because it rewrites those slots)
-    g = torch.Generator(device=dev).manual_seed(7)
-    k_new = torch.randn((T, 128), generator=g, device=dev, dtype=torch.float32)
-    c_new = torch.randn((T, 576), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
-    cw_ms = timed_mean(lambda: dsa.cache_write(db.batch, plan_t, k_new, c_new, db.kI_cache, db.kI_scale,
-                                               db.kv_cache), max(3, min(args.steps, 20)))
-    cw_bytes = T * (128 * 4 + 576 * 2 + 128 + 4 + 576 * 2)
-
-    short = None
-    if not args.no_short_prefill:
-        reps = max(3, min(args.steps, 20))
-        short = [short_prefill_mha(dev, timed_mean, reps, tf_peak, synth.workload("prefill_2048"),
-                                   "prefill_2048 (masked MHA mode): L 2048, 16 heads, k 512"),
-                 short_prefill_mha(dev, timed_mean, reps, tf_peak,
-                                   synth.custom("prefill_4k_128h", [4096], [4096], n_heads=128, topk=2048),
-                                   "masked MHA mode at the model's head count: L 4096, 128 heads, k 2048")]
-
-    # end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        pin = lambda t: t.cpu().pin_memory()
-        h_in = {"qI": pin(db.qI.view(torch.uint8)), "qI_scale": pin(db.qI_scale), "wI": pin(db.wI),
-                "q": pin(db.q), "seq_lens": pin(db.batch.seq_lens), "cu_q": pin(db.batch.cu_q),
-                "block_table": pin(db.batch.block_table)}
-        d_in = {n: torch.empty_like(t, device=dev) for n, t in h_in.items()}
-        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in h_in.values())
-        d2h = h_out.numel() * h_out.element_size()
-        batch2 = dsa.Batch(d_in["seq_lens"], d_in["cu_q"], d_in["block_table"], hb.num_pages, T, db.batch.c.max_q,
-                           hb.max_seq_len)
-        qI_d = d_in["qI"].view(torch.float8_e4m3fn)
-
-        def e2e_step():
-            for n in h_in:
-                d_in[n].copy_(h_in[n], non_blocking=True)
-            dsa.layer(batch2, qI_d, d_in["qI_scale"], d_in["wI"], db.kI_cache, db.kI_scale, d_in["q"],
-                      db.kv_cache, db.k, db.softmax_scale, out=out, ws=ws)
-            h_out.copy_(out, non_blocking=True)
-
-        for _ in range(max(args.warmup, 1)):
-            e2e_step()
-        barrier()
-        es, ee = [], []
-        for i in range(args.steps):
-            flush.fill_(i & 0xFF)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            e2e_step()
-            b.record(stream)
-            es.append(a)
-            ee.append(b)
-        barrier()
-        e_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in zip(es, ee)), dist, dev)
-        e2e = {"value": job_throughput(T, world, e_ms), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "ms_per_step": e_ms}
+        e2e = e2e_pipelined(dsa, torch, r, r.hb, dev, max(3, min(args.steps, 10)), 2, dist)
+        e2e["value"] = job_throughput(T, world, e2e["ms_per_step"])
+    hb_head = r.hb
+    del r
+    torch.cuda.empty_cache()
 
     if dist is not None:
         dist.barrier()
@@ -485,44 +612,68 @@ def main():
     if rank != 0:
         return 0
 
+    workloads = None
+    if world == 1 and not args.only_headline:
+        workloads = {wl.name: head}
+        for name in ALL_WORKLOADS:
+            if name == wl.name:
+                continue
+            rep, rr = measure_workload(dsa, torch, synth.workload(name), dev, 0, args.steps, args.warmup, flush,
+                                       sampler, peaks)
+            workloads[name] = rep
+            del rr
+            torch.cuda.empty_cache()
+
+    short = None
+    if not args.no_short_prefill:
+        reps = max(3, min(args.steps, 10))
+        short = [short_prefill_mha(dsa, torch, synth, dev, flush, reps, peaks["bf16_TFLOPs"],
+                                   synth.workload("prefill_2048"),
+                                   "prefill_2048 (masked MHA mode): L 2048, 16 heads, k 512"),
+                 short_prefill_mha(dsa, torch, synth, dev, flush, reps, peaks["bf16_TFLOPs"],
+                                   synth.custom("prefill_4k_128h", [4096], [4096], n_heads=128, topk=2048),
+                                   "masked MHA mode at the model's head count: L 4096, 128 heads, k 2048")]
+
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        rate, rows, dt = time_oracle(hb, budget_s=12.0)
+        rate, rows, dt = time_oracle(hb_head, budget_s=12.0)
         cpu = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-               "sample": f"{rows} of the {T} query rows of {wl.name} through the whole path in "
-                         f"{dt:.1f} s (float64 numpy, BLAS threads)"}
+               "sample": f"{rows} uniformly drawn of the {T} query rows of {wl.name} through the whole path in "
+                         f"{dt:.1f} s (float64 numpy, BLAS threads); rows/s estimates the whole step"}
         try:  # the same oracle on one thread, a smaller sample
             from threadpoolctl import threadpool_limits
             with threadpool_limits(limits=1):
-                r1, n1, d1 = time_oracle(hb, budget_s=4.0)
-            cpu["single_thread"] = {"value": r1, "unit": UNIT, "cores": 1,
-                                    "sample": f"{n1} query rows in {d1:.1f} s"}
+                r1, n1, d1 = time_oracle(hb_head, budget_s=4.0, seed=1)
+            cpu["single_thread"] = {"value": r1, "unit": UNIT, "cores": 1, "sample": f"{n1} query rows in {d1:.1f} s"}
         except ImportError:
             pass
 
-    launches_per_step = 3 + (1 if mla_ws_n > 0 else 0) + (1 if topk_ws_n > 0 else 0)
+    stages = head["stages"]
+    dominant = max(stages, key=lambda n: stages[n]["us"])
+    d = stages[dominant]
+    roofline = {"bound": d["bound"], "kernel": dominant, "achieved": d["achieved"], "peak": d["peak"],
+                "unit": d["unit"], "frac": d["frac"],
+                "algorithmic": d["algorithmic_flops"] if d["bound"] == "tensor" else d["algorithmic_bytes"],
+                "traffic": recorded_traffic(dominant + "_kernel", wl.name),
+                "peak_source": peaks["source"] if (d["bound"] == "hbm" or d.get("dtype") == "bf16")
+                else peaks["fp8_source"]}
+    if d["bound"] == "tensor" and d.get("dtype") == "bf16":
+        roofline["frac_of_sustained_peak"] = d["achieved"] / peaks["bf16_TFLOPs_sustained"]
+
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "layer_us": 1e3 * ms,
-        "layer_with_plan_us": 1e3 * layer_plan_ms, "plan_us": 1e3 * plan_ms, "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": ms, "layer_us": head["layer_us"],
+        "layer_with_plan_us": head["layer_with_plan_us"], "plan_us": head["plan_us"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3+bf16 (fp32 accumulate)", "data": "synthetic",
-        "config": {"workload": wl.name, "requests": wl.batch, "query_rows": T, "context": max(wl.seq_lens),
-                   "topk": wl.topk, "index_heads": wl.n_heads_index, "heads": wl.n_heads, "page_size": 64,
-                   "l2": "256 MiB flush between timed steps", "parallelism": f"{world} independent ranks",
-                   "step": "dsa_index_scores + dsa_topk + dsa_sparse_mla, batch plan computed once per batch"},
-        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "algorithmic_bytes": dom_bytes,
-                     "traffic": recorded_traffic(dominant + "_kernel", wl.name), "peak_source": peak_src},
-        "layer_roofline": {"algorithmic_bytes": total_bytes,
-                           "achieved_GBps": total_bytes / (ms / 1e3) / 1e9,
-                           "frac": total_bytes / (ms / 1e3) / 1e9 / hbm_peak},
-        "stages": stage_report,
-        "cache_write": {"us": 1e3 * cw_ms, "GBps": cw_bytes / (cw_ms / 1e3) / 1e9, "algorithmic_bytes": cw_bytes,
-                        "note": "the step before the layer, not in the step; one launch, event-timed"},
+        "config": config_of(wl, world),
+        "roofline": roofline,
+        "peaks": peaks,
+        "stages": stages,
+        "workloads": workloads,
         "short_prefill": short,
         "e2e": e2e,
         "cpu_baseline": cpu,
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": head["launches_per_step"] * args.steps,
         "clocks": sampler.summary(),
     }
     print(json.dumps(line), flush=True)

@@ -183,15 +183,22 @@ dsa_status_t dsa_layer(const dsa_batch_t* batch, const uint8_t* qI, const float*
  * they run a layer (a locked or defragmenting memory pool, allocator-free runtimes, hooks that
  * must not call cudaMalloc). Same arguments and results as dsa_layer, minus ws/ws_bytes: the
  * workspace comes from a file-scope device array of 64 MiB that every GPU loading the library
- * holds until exit. Requests needing more than that (dsa_layer_workspace_size > 64 MiB) return
- * DSA_ERR_WORKSPACE and launch nothing. Allocates nothing. The first call on a device looks up the
- * array's device address (cudaGetSymbolAddress): make it before any stream capture. All calls share
- * the array, which keeps the last call's contents; calls whose kernels overlap on the GPU race on
- * it. The plan (for dsa_status_read) lives in that array and is not exposed. */
+ * holds until exit. Arguments are checked exactly as dsa_layer checks them (same statuses); then
+ * requests needing more than 64 MiB (dsa_layer_workspace_size) return DSA_ERR_WORKSPACE and launch
+ * nothing. Allocates nothing. Every call looks up the array's device address on the current device
+ * (cudaGetSymbolAddress, host side); the first call on a device also loads the library's device
+ * code there: make it before any stream capture. All calls share the array, which keeps the last
+ * call's contents; calls whose kernels overlap on the GPU race on it. */
 dsa_status_t dsa_layer_noalloc(const dsa_batch_t* batch, const uint8_t* qI, const float* qI_scale, const float* wI,
                                int nhI, const uint8_t* kI_cache, const float* kI_scale, const void* q, int H,
                                const void* kv_cache, int k, float softmax_scale, void* out, float* lse,
                                int32_t* S_out, void* stream);
+
+/* The status word of the last dsa_layer_noalloc call on the current device (its plan lives in the
+ * static array): synchronises `stream`, returns DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE_INDEX as
+ * dsa_status_read does, and clears the word. Read it before the next dsa_layer_noalloc call, whose
+ * plan kernel rewrites the word. No counterpart on the pages. */
+dsa_status_t dsa_layer_noalloc_status_read(void* stream);
 
 const char* dsa_status_string(dsa_status_t status);
 int dsa_abi_version(void);

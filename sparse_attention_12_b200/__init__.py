@@ -40,7 +40,7 @@ class DsaBatchC(ctypes.Structure):
 
 EXPORTS = ("dsa_abi_version", "dsa_status_string", "dsa_plan_workspace_size", "dsa_plan", "dsa_status_read",
            "dsa_index_scores", "dsa_topk_workspace_size", "dsa_topk", "dsa_sparse_mla_workspace_size", "dsa_sparse_mla",
-           "dsa_layer_workspace_size", "dsa_layer", "dsa_layer_noalloc", "dsa_cache_write",
+           "dsa_layer_workspace_size", "dsa_layer", "dsa_layer_noalloc", "dsa_layer_noalloc_status_read", "dsa_cache_write",
            "dsa_masked_mha_workspace_size", "dsa_masked_mha")
 
 _lib = None
@@ -70,6 +70,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "dsa_layer_workspace_size": (SZ, [BP, I, I, I]),
         "dsa_layer": (I, [BP, P, P, P, I, P, P, P, I, P, I, ctypes.c_float, P, P, P, P, SZ, P]),
         "dsa_layer_noalloc": (I, [BP, P, P, P, I, P, P, P, I, P, I, ctypes.c_float, P, P, P, P]),
+        "dsa_layer_noalloc_status_read": (I, [P]),
         "dsa_cache_write": (I, [BP, P, P, P, P, P, P, P]),
         "dsa_masked_mha_workspace_size": (SZ, [BP, I, I]),
         "dsa_masked_mha": (I, [BP, P, P, P, P, I, P, I, ctypes.c_float, P, P, P, SZ, P]),

@@ -55,6 +55,27 @@ size_t scores_ld(const dsa_batch_t* b) {
 
 }  // namespace
 
+namespace dsa {
+
+dsa_status_t check_layer_args(const dsa_batch_t* batch, const uint8_t* qI, const float* qI_scale, const float* wI,
+                              int nhI, const uint8_t* kI_cache, const float* kI_scale, const void* q, int H,
+                              const void* kv_cache, int k, float softmax_scale, const void* out) {
+  dsa_status_t st = check_batch(batch);
+  if (st != DSA_OK) return st;
+  if (!valid_nhI(nhI)) return DSA_ERR_UNSUPPORTED;
+  if (H < 1 || H > 128 || k < 1 || k > kMaxTopK) return DSA_ERR_UNSUPPORTED;
+  if (batch->total_q == 0) return DSA_OK;
+  if (!qI || !qI_scale || !wI || !kI_cache || !kI_scale || !q || !kv_cache || !out) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(qI) || !aligned16(kI_cache) || !aligned16(kI_scale) || !aligned16(q) || !aligned16(kv_cache) ||
+      !aligned16(out))
+    return DSA_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f)) return DSA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(batch->total_q) * nhI > (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+}  // namespace dsa
+
 extern "C" {
 
 int dsa_abi_version(void) { return DSA_ABI_VERSION; }
@@ -207,17 +228,10 @@ dsa_status_t dsa_layer(const dsa_batch_t* batch, const uint8_t* qI, const float*
                        const uint8_t* kI_cache, const float* kI_scale, const void* q, int H, const void* kv_cache,
                        int k, float softmax_scale, void* out, float* lse, int32_t* S_out, void* ws, size_t ws_bytes,
                        void* stream) {
-  dsa_status_t st = check_batch(batch);
-  if (st != DSA_OK) return st;
-  if (!valid_nhI(nhI)) return DSA_ERR_UNSUPPORTED;
-  if (H < 1 || H > 128 || k < 1 || k > kMaxTopK) return DSA_ERR_UNSUPPORTED;
-  if (batch->total_q == 0) return DSA_OK;
-  if (!qI || !qI_scale || !wI || !kI_cache || !kI_scale || !q || !kv_cache || !out || !ws) return DSA_ERR_INVALID_ARG;
-  if (!aligned16(qI) || !aligned16(kI_cache) || !aligned16(kI_scale) || !aligned16(q) || !aligned16(kv_cache) ||
-      !aligned16(out) || !aligned16(ws))
-    return DSA_ERR_INVALID_ARG;
-  if (!(softmax_scale > 0.f)) return DSA_ERR_INVALID_ARG;
-  if (static_cast<int64_t>(batch->total_q) * nhI > (int64_t(1) << 31)) return DSA_ERR_UNSUPPORTED;
+  const dsa_status_t st = check_layer_args(batch, qI, qI_scale, wI, nhI, kI_cache, kI_scale, q, H, kv_cache, k,
+                                           softmax_scale, out);
+  if (st != DSA_OK || batch->total_q == 0) return st;
+  if (!ws || !aligned16(ws)) return DSA_ERR_INVALID_ARG;
   if (ws_bytes < dsa_layer_workspace_size(batch, nhI, H, k)) return DSA_ERR_WORKSPACE;
 
   const size_t T = static_cast<size_t>(batch->total_q);

@@ -93,6 +93,12 @@ DSA_HD inline PlanView plan_view(void* base, int B, int T) {
   return v;
 }
 
+// Every check dsa_layer makes before it launches, except those of the workspace (shared with
+// dsa_layer_noalloc). DSA_OK also for an empty batch with valid sizes.
+dsa_status_t check_layer_args(const dsa_batch_t* batch, const uint8_t* qI, const float* qI_scale, const float* wI,
+                              int nhI, const uint8_t* kI_cache, const float* kI_scale, const void* q, int H,
+                              const void* kv_cache, int k, float softmax_scale, const void* out);
+
 // ---- launchers (defined in the .cu files; return cudaError_t as int) ---------------------
 struct BatchDev {
   int B, T, max_q, max_seq_len, max_pages, num_pages;

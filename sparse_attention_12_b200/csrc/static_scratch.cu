@@ -7,39 +7,30 @@
 // sets, split partials) out of one file-scope device array instead.
 //
 // The array is kStaticScratchBytes (64 MiB) per device; every GPU that loads the library holds it
-// until the process exits. Its device address is looked up once per device, on that device's
-// first call, with cudaGetSymbolAddress; make that first call before any stream capture.
+// until the process exits. Its device address is looked up with cudaGetSymbolAddress on every
+// call (a host-side query; the address can change if the device's primary context is torn down
+// and created again). The first call on a device also loads the library's device code there:
+// make that first call before any stream capture.
 // All calls share the array and it keeps the last call's contents: calls whose kernels overlap
 // on the GPU (different streams, or several host threads) race on it. Nothing in it needs to
 // start at zero: the plan kernel rewrites the status word and every other region is written
-// before it is read.
+// before it is read. The plan, with the status word the kernels record run-time faults in, sits at
+// the start of the array; dsa_layer_noalloc_status_read reads (and clears) that word.
 #include <cuda_runtime.h>
-
-#include <mutex>
 
 #include "dsa_internal.h"
 
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(64) << 20;
-constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-std::mutex g_scratch_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
-
 // Device address of g_static_scratch on the current device (nullptr on failure).
 void* scratch_for_current_device() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_ptr[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess) return nullptr;
-    g_scratch_ptr[dev] = ptr;
-  }
-  return g_scratch_ptr[dev];
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess) return nullptr;
+  return ptr;
 }
 
 }  // namespace
@@ -48,15 +39,21 @@ extern "C" dsa_status_t dsa_layer_noalloc(const dsa_batch_t* batch, const uint8_
                                           const float* wI, int nhI, const uint8_t* kI_cache, const float* kI_scale,
                                           const void* q, int H, const void* kv_cache, int k, float softmax_scale,
                                           void* out, float* lse, int32_t* S_out, void* stream) {
-  if (!batch) return DSA_ERR_INVALID_ARG;
-  if (batch->total_q == 0 && batch->num_requests >= 0) return DSA_OK;
+  // the same argument checks, in the same order, as dsa_layer; then the size limit
+  const dsa_status_t st = dsa::check_layer_args(batch, qI, qI_scale, wI, nhI, kI_cache, kI_scale, q, H, kv_cache,
+                                                k, softmax_scale, out);
+  if (st != DSA_OK || batch->total_q == 0) return st;
   const size_t need = dsa_layer_workspace_size(batch, nhI, H, k);
-  if (need == 0)  // invalid sizes: let dsa_layer report which status applies
-    return dsa_layer(batch, qI, qI_scale, wI, nhI, kI_cache, kI_scale, q, H, kv_cache, k, softmax_scale, out, lse,
-                     S_out, nullptr, 0, stream);
+  if (need == 0) return DSA_ERR_INVALID_ARG;  // unreachable once the checks above passed
   if (need > kStaticScratchBytes) return DSA_ERR_WORKSPACE;
   void* ws = scratch_for_current_device();
   if (!ws) return DSA_ERR_CUDA;
   return dsa_layer(batch, qI, qI_scale, wI, nhI, kI_cache, kI_scale, q, H, kv_cache, k, softmax_scale, out, lse,
                    S_out, ws, kStaticScratchBytes, stream);
+}
+
+extern "C" dsa_status_t dsa_layer_noalloc_status_read(void* stream) {
+  void* ws = scratch_for_current_device();
+  if (!ws) return DSA_ERR_CUDA;
+  return dsa_status_read(ws, stream);
 }

@@ -13,12 +13,17 @@ Workload shapes follow the DSA configuration on the pages:
     indexer key per position, per-query head weights w_t, causal visibility j <= t.
 Page size 64 is the paged-cache granularity the serving commands on the pages use.
 
-Random draws use numpy's PCG64 seeded with SeedSequence([seed, workload_id]).
+Random draws use numpy's PCG64: the page permutation and the needles from SeedSequence([seed,
+workload_id]), every large array from SeedSequence([seed, workload_id, array tag]) in blocks of
+whole rows, each block from its own spawned child (drawn on host threads; the values do not
+depend on the thread count).
 """
 from __future__ import annotations
 
 import dataclasses
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 from typing import Optional
 
 import numpy as np
@@ -116,10 +121,17 @@ def quantize_e4m3_per_token(x: np.ndarray):
     x = np.asarray(x, dtype=np.float32)
     lead = x.shape[0]
     flat = x.reshape(lead, -1)
-    amax = np.abs(flat).max(axis=1)
-    scale = np.where(amax > 0, amax / np.float32(FP8_MAX), np.float32(1.0)).astype(np.float32)
-    y = np.clip(flat / scale[:, None], -FP8_MAX, FP8_MAX).astype(np.float32)
-    codes = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    codes = np.empty(flat.shape, np.uint8)
+    scale = np.empty(lead, np.float32)
+
+    def work(lo, hi):
+        amax = np.abs(flat[lo:hi]).max(axis=1)
+        sc = np.where(amax > 0, amax / np.float32(FP8_MAX), np.float32(1.0)).astype(np.float32)
+        y = np.clip(flat[lo:hi] / sc[:, None], -FP8_MAX, FP8_MAX).astype(np.float32)
+        codes[lo:hi] = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        scale[lo:hi] = sc
+
+    _row_blocks(work, lead, max(1, _BLOCK_ELEMS // max(1, flat.shape[1])))
     return codes.reshape(x.shape), scale
 
 
@@ -182,14 +194,46 @@ class Batch:
         return req, pos
 
 
-def _normal_bf16(rng: np.random.Generator, shape, chunk_rows: int = 1 << 14) -> np.ndarray:
-    """N(0,1) draws stored as bf16 bits, generated in row chunks to bound host memory."""
-    out = np.empty(shape, np.uint16)
-    flat = out.reshape(shape[0], -1)
-    for lo in range(0, shape[0], chunk_rows):
-        hi = min(shape[0], lo + chunk_rows)
-        flat[lo:hi] = f32_to_bf16_bits(rng.standard_normal((hi - lo, flat.shape[1]), dtype=np.float32))
+# Large arrays are drawn in blocks of whole leading rows (about _BLOCK_ELEMS values each), every
+# block from its own child of the array's SeedSequence, on a pool of host threads. The values do
+# not depend on the number of threads.
+_BLOCK_ELEMS = 1 << 22
+
+
+def _row_blocks(fn, n_rows: int, rows_per_block: int):
+    """fn(lo, hi) over consecutive row blocks, on a thread pool (numpy and torch release the GIL)."""
+    spans = [(lo, min(n_rows, lo + rows_per_block)) for lo in range(0, n_rows, rows_per_block)]
+    if len(spans) <= 1:
+        for lo, hi in spans:
+            fn(lo, hi)
+        return
+    workers = max(1, min(32, len(os.sched_getaffinity(0)), len(spans)))
+    with ThreadPoolExecutor(workers) as ex:
+        for f in [ex.submit(fn, lo, hi) for lo, hi in spans]:
+            f.result()
+
+
+def _normal(ss: np.random.SeedSequence, shape, as_bf16: bool) -> np.ndarray:
+    """N(0,1) draws of `shape`, float32 or stored as bf16 bits."""
+    out = np.empty(shape, np.uint16 if as_bf16 else np.float32)
+    n_rows = int(shape[0])
+    flat = out.reshape(n_rows, -1)
+    rows_per_block = max(1, _BLOCK_ELEMS // max(1, flat.shape[1]))
+    children = ss.spawn((n_rows + rows_per_block - 1) // rows_per_block)
+
+    def work(lo, hi):
+        g = np.random.Generator(np.random.PCG64(children[lo // rows_per_block]))
+        if as_bf16:
+            flat[lo:hi] = f32_to_bf16_bits(g.standard_normal((hi - lo, flat.shape[1]), dtype=np.float32))
+        else:
+            g.standard_normal((hi - lo, flat.shape[1]), dtype=np.float32, out=flat[lo:hi])
+
+    _row_blocks(work, n_rows, rows_per_block)
     return out
+
+
+def _seq(seed: int, wl: "Workload", tag: int) -> np.random.SeedSequence:
+    return np.random.SeedSequence([seed, wl.wid, tag])
 
 
 def make_batch(wl: Workload, seed: int = 0, extra_pages: int = 0) -> Batch:
@@ -215,10 +259,10 @@ def make_batch(wl: Workload, seed: int = 0, extra_pages: int = 0) -> Batch:
 
     nhI, H = wl.n_heads_index, wl.n_heads
     # indexer queries and head weights
-    qI_f = rng.standard_normal((T, nhI, D_INDEX), dtype=np.float32)
-    wI = (rng.standard_normal((T, nhI), dtype=np.float32) / np.float32(math.sqrt(nhI))).astype(np.float32)
+    qI_f = _normal(_seq(seed, wl, 1), (T, nhI, D_INDEX), False)
+    wI = (_normal(_seq(seed, wl, 2), (T, nhI), False) / np.float32(math.sqrt(nhI))).astype(np.float32)
     # indexer keys, one per logical position, float before quantisation
-    kI_f = rng.standard_normal((P, PAGE, D_INDEX), dtype=np.float32)
+    kI_f = _normal(_seq(seed, wl, 3), (P, PAGE, D_INDEX), False)
 
     # needles: k_j <- 0.8 * q_{t, r*} + 0.2 * noise, r* = argmax_r w_tr
     needles = []
@@ -259,8 +303,8 @@ def make_batch(wl: Workload, seed: int = 0, extra_pages: int = 0) -> Batch:
     kI_cache = kI_codes.reshape(P, PAGE, D_INDEX)
     kI_scale = kI_scale.reshape(P, PAGE)
 
-    q = _normal_bf16(rng, (T, H, D_LATENT), chunk_rows=max(1, (1 << 22) // (H * D_LATENT)))
-    kv_cache = _normal_bf16(rng, (P, PAGE, D_LATENT), chunk_rows=max(1, (1 << 22) // (PAGE * D_LATENT)))
+    q = _normal(_seq(seed, wl, 4), (T, H, D_LATENT), True)
+    kv_cache = _normal(_seq(seed, wl, 5), (P, PAGE, D_LATENT), True)
     return Batch(wl, qI, qI_scale, wI, kI_cache, kI_scale, q, kv_cache, block_table,
                  seq_lens, cu_q, needles)
 
@@ -284,12 +328,10 @@ class MhaInputs:
 
 def make_mha_inputs(wl: Workload, seed: int = 0) -> MhaInputs:
     assert tuple(wl.seq_lens) == tuple(wl.q_per_req), "the masked MHA mode takes whole prefills"
-    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, wl.wid, 7])))
     T, H = wl.total_q, wl.n_heads
-    rows = max(1, (1 << 22) // (H * D_QK_MHA))
-    q = _normal_bf16(rng, (T, H, D_QK_MHA), chunk_rows=rows)
-    k = _normal_bf16(rng, (T, H, D_QK_MHA), chunk_rows=rows)
-    v = _normal_bf16(rng, (T, H, D_V_MHA), chunk_rows=rows)
+    q = _normal(np.random.SeedSequence([seed, wl.wid, 7, 0]), (T, H, D_QK_MHA), True)
+    k = _normal(np.random.SeedSequence([seed, wl.wid, 7, 1]), (T, H, D_QK_MHA), True)
+    v = _normal(np.random.SeedSequence([seed, wl.wid, 7, 2]), (T, H, D_V_MHA), True)
     return MhaInputs(q, k, v)
 
 

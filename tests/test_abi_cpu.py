@@ -46,11 +46,18 @@ def test_abi_version_and_strings(lib):
 
 FAKE = 1 << 20  # an aligned, never-dereferenced "device" address: validation must fail first
 
+# The validation tests below pass made-up device addresses that the host-side checks must reject
+# before anything launches. They run only where no GPU can be reached, so that a change in the
+# order of the checks can never send a kernel to those addresses.
+no_gpu = pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                            reason="made-up device addresses: run where no GPU is reachable")
+
 
 def batch(B=2, T=3, max_q=2, max_seq_len=300, max_pages=5, num_pages=10):
     return dsa.DsaBatchC(B, T, max_q, max_seq_len, max_pages, num_pages, FAKE, FAKE, FAKE)
 
 
+@no_gpu
 def test_plan_rejects_bad_arguments(lib):
     b = batch()
     n = lib.dsa_plan_workspace_size(ctypes.byref(b), 64)
@@ -75,6 +82,7 @@ def test_empty_batch_is_a_no_op(lib):
                          None, None, None, 0, None) == 0
 
 
+@no_gpu
 def test_index_scores_validation(lib):
     b = batch()
     call = lambda **kw: lib.dsa_index_scores(
@@ -88,6 +96,7 @@ def test_index_scores_validation(lib):
     assert call(scores=None) == 1
 
 
+@no_gpu
 def test_cache_write_validation(lib):
     b = batch()
     call = lambda **kw: lib.dsa_cache_write(ctypes.byref(b), kw.get("plan", FAKE), kw.get("k", FAKE), kw.get("c", FAKE),
@@ -100,6 +109,7 @@ def test_cache_write_validation(lib):
     assert lib.dsa_cache_write(ctypes.byref(empty), None, None, None, None, None, None, None) == 0
 
 
+@no_gpu
 def test_topk_and_mla_validation(lib):
     b = batch()
     assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE, 384, 0, FAKE, None, 0, None) == 2
@@ -130,6 +140,7 @@ def test_topk_and_mla_validation(lib):
     assert mla(ws_bytes=need - 1) == 3
 
 
+@no_gpu
 def test_layer_workspace_accounting(lib):
     b = batch()
     n = lib.dsa_layer_workspace_size(ctypes.byref(b), 64, 128, 2048)
@@ -144,6 +155,7 @@ def test_layer_workspace_accounting(lib):
     assert lib.dsa_layer(*args[:4], 40, *args[5:], n, None) == 2
 
 
+@no_gpu
 def test_masked_mha_validation(lib):
     b = batch()
     need = lib.dsa_masked_mha_workspace_size(ctypes.byref(b), 16, 512)
@@ -168,3 +180,33 @@ def test_masked_mha_validation(lib):
     empty = dsa.DsaBatchC(0, 0, 0, 0, 0, 0, None, None, None)
     assert lib.dsa_masked_mha(ctypes.byref(empty), None, None, None, None, 16, None, 512, 0.07, None, None, None, 0,
                               None) == 0
+
+
+@no_gpu
+def test_noalloc_checks_arguments_like_layer(lib):
+    """dsa_layer_noalloc returns what dsa_layer returns for every argument error, and only then
+    applies its size limit (nothing launches in any of these calls)."""
+    empty = dsa.DsaBatchC(0, 0, 0, 0, 0, 0, None, None, None)
+    for nhI, H, k in [(48, 128, 2048), (64, 0, 2048), (64, 128, 0), (64, 128, 2048)]:
+        want = lib.dsa_layer(ctypes.byref(empty), None, None, None, nhI, None, None, None, H, None, k, 0.07, None,
+                             None, None, None, 0, None)
+        got = lib.dsa_layer_noalloc(ctypes.byref(empty), None, None, None, nhI, None, None, None, H, None, k, 0.07,
+                                    None, None, None, None)
+        assert got == want == (0 if (nhI, H, k) == (64, 128, 2048) else 2)
+    # 40000 query rows x 2048 positions of fp32 scores alone need 312 MiB of workspace
+    big = dsa.DsaBatchC(1, 40000, 40000, 40000, 625, 700, FAKE, FAKE, FAKE)
+    assert lib.dsa_layer_workspace_size(ctypes.byref(big), 64, 128, 2048) > (64 << 20)
+
+    def noalloc(**kw):
+        return lib.dsa_layer_noalloc(ctypes.byref(big), kw.get("qI", FAKE), FAKE, FAKE, 64, FAKE, FAKE, FAKE, 128,
+                                     FAKE, 2048, ctypes.c_float(kw.get("scale", 0.07)), kw.get("out", FAKE), None,
+                                     None, None)
+
+    def layer(**kw):
+        return lib.dsa_layer(ctypes.byref(big), kw.get("qI", FAKE), FAKE, FAKE, 64, FAKE, FAKE, FAKE, 128, FAKE, 2048,
+                             ctypes.c_float(kw.get("scale", 0.07)), kw.get("out", FAKE), None, None, FAKE, 1 << 40,
+                             None)
+
+    for bad in ({"qI": None}, {"out": None}, {"qI": FAKE + 4}, {"scale": 0.0}):
+        assert noalloc(**bad) == layer(**bad) == 1, bad
+    assert noalloc() == 3  # valid arguments, above the 64 MiB static array: DSA_ERR_WORKSPACE

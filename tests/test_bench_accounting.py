@@ -54,3 +54,45 @@ def test_causal_prefill_counts_visible_positions_only():
     assert w["index_scores"][1] == vis * 2 * 16 * 128
     assert w["sparse_mla"][1] == sel * (2 * 16 * 576 + 2 * 16 * 512)
     assert w["topk"][0] == vis * 4 + L * 64 * 4
+    # the latent rows once (the whole cache of this request is named), indices, queries, output
+    assert w["sparse_mla"][0] == L * 1152 + sel * 4 + L * 16 * 576 * 2 + L * 16 * 512 * 2
+
+
+def test_mtp_rows_counted_once_per_request_at_most():
+    # two queries of one request: at most 2k distinct rows, never more than the request holds
+    hb = _fake_batch([131072, 3000], [2, 2], nhI=64, H=128, k=2048)
+    w = bench.algorithmic(hb)
+    rows = 2 * 2048 + 3000                   # request 1 holds 3000 positions, both of its rows see them all
+    assert w["sparse_mla"][0] == rows * 1152 + (2 * 2048 + 2 * 2048) * 4 + 4 * 128 * (576 + 512) * 2
+
+
+PEAKS = {"hbm_GBps": 6549.8, "bf16_TFLOPs": 1645.6, "fp8_TFLOPs": 3291.2}
+
+
+def test_stage_bound_is_the_longer_roofline_time():
+    # decode_64x16k's indexer: 124 FLOP per byte, below the FP8 ridge (~502) -> HBM-bound
+    hb = _fake_batch([16384] * 64, [1] * 64, nhI=64, H=128, k=2048)
+    w = bench.algorithmic(hb)
+    r = bench.stage_roofline("index_scores", *w["index_scores"], 50.0, PEAKS)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert abs(r["roofline_us"] - w["index_scores"][0] / 6549.8e9 * 1e6) < 1e-9
+    assert abs(r["frac"] - r["roofline_us"] / 50.0) < 1e-12
+    # a causal prefill's indexer: FLOPs grow with L^2, bytes with L -> FP8 tensor-bound
+    hb = _fake_batch([32768], [32768], nhI=64, H=128, k=2048)
+    w = bench.algorithmic(hb)
+    r = bench.stage_roofline("index_scores", *w["index_scores"], 8000.0, PEAKS)
+    assert r["bound"] == "tensor" and r["dtype"] == "fp8" and r["peak"] == 3291.2
+    assert abs(r["achieved"] - w["index_scores"][1] / 8000e-6 / 1e12) < 1e-6
+    # its sparse MLA at bf16, and the top-k (no contraction) always against HBM
+    r = bench.stage_roofline("sparse_mla", *w["sparse_mla"], 30000.0, PEAKS)
+    assert r["bound"] == "tensor" and r["dtype"] == "bf16" and r["peak"] == 1645.6
+    r = bench.stage_roofline("topk", *w["topk"], 3000.0, PEAKS)
+    assert r["bound"] == "hbm" and "tensor_frac" not in r
+
+
+def test_both_arms_describe_the_same_config():
+    from sparse_attention_12_b200 import synth
+    wl = synth.workload("prefill_32k")
+    c = bench.config_of(wl, 1)
+    assert c["workload"] == "prefill_32k" and c["query_rows"] == 32768 and c["context"] == 32768
+    assert set(c) >= {"workload", "page_size", "l2", "parallelism", "step"}
