@@ -46,7 +46,7 @@
 extern "C" {
 #endif
 
-#define DSA_ABI_VERSION 3
+#define DSA_ABI_VERSION 4
 #define DSA_PAGE_SIZE 64   /* positions per cache page */
 #define DSA_D_INDEX 128    /* indexer head width d_h^I */
 #define DSA_D_LATENT 576   /* latent width: 512 + 64 rope */
@@ -61,7 +61,8 @@ typedef enum {
   DSA_ERR_WORKSPACE = 3,    /* workspace smaller than *_workspace_size */
   DSA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
   DSA_ERR_TIMEOUT = 5,      /* a kernel wait gave up (read back by dsa_status_read) */
-  DSA_ERR_DEVICE_INDEX = 6  /* a kernel met an index outside its buffers (dsa_status_read) */
+  DSA_ERR_DEVICE_INDEX = 6, /* a kernel met an index outside its buffers (dsa_status_read) */
+  DSA_ERR_DEVICE_VALUE = 7  /* a kernel met a non-finite input value (dsa_status_read) */
 } dsa_status_t;
 
 /* A ragged batch of requests. Shared by every call. */
@@ -85,7 +86,8 @@ size_t dsa_plan_workspace_size(const dsa_batch_t* batch, int nhI);
 dsa_status_t dsa_plan(const dsa_batch_t* batch, int nhI, void* plan, size_t plan_bytes, void* stream);
 
 /* Synchronises `stream`, then returns the status word the kernels of the last calls that used
- * `plan` recorded (DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE_INDEX) and clears it. */
+ * `plan` recorded (DSA_OK, DSA_ERR_TIMEOUT, DSA_ERR_DEVICE_INDEX or DSA_ERR_DEVICE_VALUE; the first of
+ * these when several were recorded) and clears it. */
 dsa_status_t dsa_status_read(void* plan, void* stream);
 
 /* ---- writing new positions into the caches (the step before step 1) ----------------------
@@ -99,9 +101,11 @@ dsa_status_t dsa_status_read(void* plan, void* stream);
  * indexer key as FP8 + a 4-byte scale, both paged; "DeepSeek Sparse Attention：从 SWA 到稀疏
  * Attention 计算", Lightning Indexer section: one shared indexer key per position in its own key
  * cache.) The plan must be made for this batch (dsa_plan).
- * k_new f32 [T, 128] (finite), c_new bf16 [T, 576]; caches as for dsa_index_scores / dsa_sparse_mla.
+ * k_new f32 [T, 128], c_new bf16 [T, 576]; caches as for dsa_index_scores / dsa_sparse_mla.
  * A page id outside [0, num_pages) is recorded as DSA_ERR_DEVICE_INDEX (dsa_status_read) and its
- * row is skipped. */
+ * row is skipped. A key with an infinite or NaN element has no FP8 encoding (it would store e4m3 NaN
+ * codes): it is recorded as DSA_ERR_DEVICE_VALUE and its row is skipped (neither cache is written
+ * there). The latent row is copied as given. */
 dsa_status_t dsa_cache_write(const dsa_batch_t* batch, const void* plan, const float* k_new, const void* c_new,
                              uint8_t* kI_cache, float* kI_scale, void* kv_cache, void* stream);
 
@@ -113,7 +117,9 @@ dsa_status_t dsa_cache_write(const dsa_batch_t* batch, const void* plan, const f
  * kI_scale f32  [P, 64]         s^k per cached position
  * scores   f32  [T, ld]         out: I_tj for j <= p; -inf for p < j < min(ld, 128*ceil((p+1)/128));
  *                               other entries untouched. ld >= max_seq_len, ld % 4 == 0.
- * Runs as an FP8 tcgen05 GEMM (keys x query-heads) with ReLU, w and the head sum in the epilogue. */
+ * Runs as an FP8 tcgen05 GEMM (keys x query-heads) with ReLU, w and the head sum in the epilogue.
+ * The caches must hold no e4m3 NaN codes (0x7F, 0xFF; dsa_cache_write never writes them): scores
+ * computed from them are undefined. */
 dsa_status_t dsa_index_scores(const dsa_batch_t* batch, const void* plan, const uint8_t* qI,
                               const float* qI_scale, const float* wI, int nhI, const uint8_t* kI_cache,
                               const float* kI_scale, float* scores, int64_t ld, void* stream);
@@ -122,8 +128,9 @@ dsa_status_t dsa_index_scores(const dsa_batch_t* batch, const void* plan, const 
  * scores f32 [T, ld] as written by dsa_index_scores (row t read at j <= p only); ld % 4 == 0,
  *        ld >= max_seq_len. max_seq_len <= 262144 (else DSA_ERR_UNSUPPORTED).
  * S      int32 [T, k] out: the min(k, p+1) positions with the largest scores, followed by -1.
- *        Among equal scores the smaller position wins. Selected positions are listed in
- *        increasing position order. 1 <= k <= 4096.
+ *        Among equal scores the smaller position wins; -0 equals +0; a NaN score ranks below every
+ *        other score (-inf included). Selected positions are listed in increasing position order.
+ *        1 <= k <= 4096.
  * ws/ws_bytes: dsa_topk_workspace_size bytes (0 when max_seq_len <= 32768): rows longer than 32768
  *        positions select per slice of 32768 first, then among the slices' winners. */
 size_t dsa_topk_workspace_size(const dsa_batch_t* batch, int k);

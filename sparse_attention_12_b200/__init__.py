@@ -23,7 +23,8 @@ D_QK_MHA = 192
 D_V_MHA = 128
 
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported size", 3: "workspace too small", 4: "CUDA error",
-          5: "a kernel wait timed out", 6: "a kernel met an out-of-range index"}
+          5: "a kernel wait timed out", 6: "a kernel met an out-of-range index",
+          7: "a kernel met a non-finite input value"}
 
 
 class DsaError(RuntimeError):

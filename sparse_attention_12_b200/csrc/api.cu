@@ -89,6 +89,7 @@ const char* dsa_status_string(dsa_status_t s) {
     case DSA_ERR_CUDA: return "CUDA error";
     case DSA_ERR_TIMEOUT: return "a kernel wait timed out";
     case DSA_ERR_DEVICE_INDEX: return "a kernel met an out-of-range index";
+    case DSA_ERR_DEVICE_VALUE: return "a kernel met a non-finite input value";
   }
   return "unknown status";
 }
@@ -116,6 +117,7 @@ dsa_status_t dsa_status_read(void* plan, void* stream) {
   if (word != 0 && cudaMemset(plan, 0, sizeof(word)) != cudaSuccess) return DSA_ERR_CUDA;
   if (word & kDevErrTimeout) return DSA_ERR_TIMEOUT;
   if (word & kDevErrIndex) return DSA_ERR_DEVICE_INDEX;
+  if (word & kDevErrValue) return DSA_ERR_DEVICE_VALUE;
   return DSA_OK;
 }
 

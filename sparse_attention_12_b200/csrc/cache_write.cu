@@ -44,6 +44,12 @@ __global__ void __launch_bounds__(32 * kRowsPerBlock)
 
   // indexer key: lane l holds elements 4l .. 4l+3
   const float4 x = __ldg(reinterpret_cast<const float4*>(k_new + static_cast<int64_t>(t) * kDIdx) + lane);
+  // a non-finite key has no FP8 encoding (it would store NaN codes): the row is not written
+  const bool finite = isfinite(x.x) && isfinite(x.y) && isfinite(x.z) && isfinite(x.w);
+  if (!__all_sync(0xffffffffu, finite)) {
+    if (lane == 0) report_error(status, kDevErrValue);
+    return;
+  }
   const float m = fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w)));
   // non-negative floats order like their bit patterns
   const float amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(m)));

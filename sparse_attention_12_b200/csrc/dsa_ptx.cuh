@@ -85,7 +85,10 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t pa
 // Wait for the phase of `bar` with the given parity to complete. Gives up after ~kWaitLimitNs
 // (or as soon as another CTA reported an error), records `code` in the status word and
 // returns false. Every pipeline wait in this library goes through here.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
+#ifndef DSA_WAIT_LIMIT_NS
+#define DSA_WAIT_LIMIT_NS 2000000000ull  // 2 s: far above any legitimate wait
+#endif
+constexpr uint64_t kWaitLimitNs = DSA_WAIT_LIMIT_NS;
 static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, uint32_t* status, uint32_t code) {
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
@@ -93,6 +96,18 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parit
     if (error_seen(status)) return false;
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       report_error(status, code);
+      return false;
+    }
+  }
+}
+// Wait for a phase whatever the status word says, still bounded by kWaitLimitNs: a CTA that gives
+// up after an error uses it to let its own copies and MMAs land before it leaves.
+static __device__ __noinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, uint32_t* status) {
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (mbar_try_wait_suspend(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      report_error(status, kDevErrTimeout);
       return false;
     }
   }
@@ -157,6 +172,25 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
+}
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+// loads, reductions and atomics on a (possibly remote) shared::cluster address
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_cluster_add_u32(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t atom_cluster_add_u32(uint32_t addr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v) : "memory");
+  return old;
 }
 // shared::cluster address of the variable at local shared address `local` in CTA `rank`
 __device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {

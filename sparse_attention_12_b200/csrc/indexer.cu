@@ -30,6 +30,16 @@
 #include "dsa_internal.h"
 #include "dsa_ptx.cuh"
 
+#ifdef DSA_TEST_FAULTS
+// Test-only build (never the product library): a switch that makes every indexer CTA leave the
+// keys of its first tile unloaded, so that the MMA issuer's bounded wait runs out and the kernel
+// must record DSA_ERR_TIMEOUT, let its other copies land, free TMEM and return.
+__device__ int g_test_fault = 0;
+extern "C" int dsa_test_set_fault(int code) {
+  return static_cast<int>(cudaMemcpyToSymbol(g_test_fault, &code, sizeof(code)));
+}
+#endif
+
 namespace dsa {
 namespace {
 
@@ -54,7 +64,7 @@ struct IdxSmem {
   static constexpr int kSq = kScale + kScaleSlots * kIdxTileKeys * 4;  // float [2][16]
   static constexpr int kMeta = kSq + 2 * 16 * 4;                  // GroupMeta [2]
   static constexpr int kBars = kMeta + 2 * 16;                    // uint64 barriers
-  static constexpr int kNumBars = 2 * kMaxStages + 4 + 2 * kMaxAcc + 2 * kScaleSlots;
+  static constexpr int kNumBars = 2 * kMaxStages + 4 + 2 * kMaxAcc + 2 * kScaleSlots + 1;
   static constexpr int kTmemSlot = kBars + kNumBars * 8;
   static constexpr int kFixed = (kTmemSlot + 16 + 1023) / 1024 * 1024;  // query buffers start here
   static constexpr int kLimit = 232448 - 1024;  // 227 KB less the slack for the 1024-byte alignment
@@ -125,6 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* tempty = tfull + kMaxAcc;
   uint64_t* sfull = tempty + kMaxAcc;
   uint64_t* sempty = sfull + kScaleSlots;
+  uint64_t* mdone = sempty + kScaleSlots;  // the MMA issuer's last commit (drained before TMEM is freed)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + IdxSmem::kTmemSlot);
 
   const int warp = warp_id(), lane = lane_id();
@@ -146,6 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], kEpiWarps);
     }
+    mbar_init(mdone, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -179,6 +191,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int pg_cache = 0, pg_next = 0;  // this window's page ids and the next window's (prefetched)
       bool ok = true;
       int s = 0, s_par = 1, c = 0, c_par = 1;  // ring positions of tile it and the parity to wait for
+      int issued = 0, q_issued = 0;            // key tiles and query boxes whose loads went out
+      int skipped = -1;                        // a key tile left unloaded by the test-only fault switch
       for (int u = u0, it = 0; u < u1 && ok; ++u, ++it) {
         const bool newg = (u == u0) || (u == gend);
         if (u == gend) {
@@ -207,6 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(base + IdxSmem::kFixed + qb * p.qbytes, &qmap, 0, gm.row0 * NHI, &qfull[qb]);
           }
           ++qcount;
+          q_issued = qcount;
           pg_base = -1;
         }
         const int kt = u - gstart;
@@ -233,7 +248,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int p_last = gm.pos0 + gm.nq - 1;
         const bool v1 = (lp0 + 1) * kPage <= p_last;
         const int q0 = min(max(pg0, 0), p.bd.num_pages - 1), q1 = min(max(pg1, 0), p.bd.num_pages - 1);
-        if (lane == 0) {
+#ifdef DSA_TEST_FAULTS
+        const bool skip = g_test_fault == 1 && it == 0;  // this tile's keys never arrive
+#else
+        constexpr bool skip = false;
+#endif
+        if (skip) skipped = it;
+        if (lane == 0 && !skip) {
           if (pg0 < 0 || pg0 >= p.bd.num_pages || (v1 && (pg1 < 0 || pg1 >= p.bd.num_pages)))
             report_error(p.status, kDevErrIndex);
           uint8_t* dst = base + IdxSmem::kFixed + 2 * p.qbytes + s * kStageBytes;
@@ -241,6 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(dst, &kmap, 0, q0 * kPage, &kfull[s]);
           if (v1) tma_load_2d(dst + kPage * kDIdx, &kmap, 0, q1 * kPage, &kfull[s]);
         }
+        issued = it + 1;
         // s^k of the tile's 128 keys: 16 bytes per lane (lanes 0..15 page 0, 16..31 page 1)
         cp_async_16(smem_u32(g_scale + c * kIdxTileKeys + 4 * lane),
                     p.kI_scale + static_cast<int64_t>(lane < 16 ? q0 : q1) * kPage + 4 * (lane & 15));
@@ -249,6 +271,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (++c == kScaleSlots) c = 0, c_par ^= 1;
       }
       asm volatile("cp.async.wait_all;" ::: "memory");
+      // no copy may still be landing when the CTA exits, also after an error: the last loads of
+      // every key stage and query buffer (already complete in a run without errors)
+      if (lane == 0) {
+        for (int j = max(0, issued - p.nstages); j < issued; ++j)
+          if (j != skipped) mbar_drain(&kfull[j % p.nstages], (j / p.nstages) & 1, p.status);
+        for (int j = max(0, q_issued - 2); j < q_issued; ++j) mbar_drain(&qfull[j & 1], (j >> 1) & 1, p.status);
+      }
+      __syncwarp();
     } else if (warp == 1) {
       // ---------------- MMA issuer ----------------
       if (lane == 0) {
@@ -287,6 +317,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&tfull[a]);
           if (u + 1 == gend || u + 1 == u1) mma_commit(&qempty[qb]);
         }
+        // every MMA this thread issued has completed before TMEM is freed (also after an error)
+        mma_commit(mdone);
+        mbar_drain(mdone, 0, p.status);
       }
       __syncwarp();
     } else {

@@ -95,7 +95,8 @@ enum : int {
   B_RED = B_PVDONE + 2,        // [2][4] partial maxima of one quadrant written (kSubs warps)
   B_LEND = B_RED + 8,          // [4]  partial sums of one quadrant written (kSubs warps)
   B_OFINAL = B_LEND + 4,       // 1    MMA -> epilogue after the last P V
-  B_COUNT = B_OFINAL + 1
+  B_MDONE = B_OFINAL + 1,      // 1    the MMA issuer's last commit (drained before TMEM is freed)
+  B_COUNT = B_MDONE + 1
 };
 static_assert(B_COUNT <= Smem::kNumBars, "barrier space");
 
@@ -187,6 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 8; ++i) mbar_init(&bar[B_RED + i], kSubs);
     for (int i = 0; i < 4; ++i) mbar_init(&bar[B_LEND + i], kSubs);
     mbar_init(&bar[B_OFINAL], 1);
+    mbar_init(&bar[B_MDONE], 1);
     fence_barrier_init();
     tma_prefetch_desc(&qmap);
     tma_prefetch_desc(&kmap);
@@ -233,6 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_3d(base + Smem::kQ + blk * kBlk, &qmap, 64 * blk, h, row0 + q0, &bar[B_QFULL]);
       }
       bool ok = true;
+      int issued = 0;  // tiles whose loads went out
       for (int i = 0; i < nkt && ok; ++i) {
         const int s = i & 1;
         ok = mbar_wait(&empty[s], ((i >> 1) & 1) ^ 1, p.status, kDevErrTimeout);
@@ -240,12 +243,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&full[s], nblk * kBlk);
         for (int blk = 0; blk < nblk; ++blk)
           tma_load_3d(ring + (s * nblk + blk) * kBlk, map, 64 * blk, h, row0 + i * kTile, &full[s]);
+        issued = i + 1;
       }
-      // no copy may still be landing when the CTA exits
-      if (is_k) mbar_wait(&bar[B_QFULL], 0, p.status, kDevErrTimeout);
-      if (ok)
-        for (int i = max(0, nkt - kStages); i < nkt; ++i)
-          mbar_wait(&full[i & 1], (i >> 1) & 1, p.status, kDevErrTimeout);
+      // no copy may still be landing when the CTA exits, also after an error
+      if (is_k) mbar_drain(&bar[B_QFULL], 0, p.status);
+      for (int i = max(0, issued - kStages); i < issued; ++i) mbar_drain(&full[i & 1], (i >> 1) & 1, p.status);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -294,6 +296,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // S buffer s was read by the softmax of tile i before it signalled P(i)
         if (i + 2 < nkt) ok = issue_qk(i + 2);
       }
+      // every MMA this thread issued has completed before TMEM is freed (also after an error)
+      mma_commit(&bar[B_MDONE]);
+      mbar_drain(&bar[B_MDONE], 0, p.status);
     }
     __syncwarp();
   } else {

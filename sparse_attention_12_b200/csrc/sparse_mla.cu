@@ -141,7 +141,9 @@ enum : int {
   B_ODONE = B_OREADY + 2,           // 1    MMA -> correction warps (once per tile)
   B_OFINAL = B_ODONE + 1,           // 1    MMA -> epilogue (once, after the last tile)
   B_STATS = B_OFINAL + 1,           // 1    S-CTA softmax -> O-CTA epilogue (128 remote arrivals)
-  B_COUNT = B_STATS + 1
+  // both
+  B_MDONE = B_STATS + 1,            // 1    the MMA issuer's last commit (drained before TMEM is freed)
+  B_COUNT = B_MDONE + 1
 };
 static_assert(B_COUNT <= Smem::kNumBars, "barrier space");
 
@@ -213,6 +215,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&bar[B_OFINAL], 1);
       mbar_init(&bar[B_STATS], 128);
     }
+    mbar_init(&bar[B_MDONE], 1);
     fence_barrier_init();
     tma_prefetch_desc(&qmap);
   }
@@ -354,12 +357,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (!ok) break;
           mma_commit(&bar[B_SFULL + sb]);
         }
+        // every MMA this thread issued has completed before TMEM is freed (also after an error)
+        mma_commit(&bar[B_MDONE]);
+        mbar_drain(&bar[B_MDONE], 0, p.status);
       }
       __syncwarp();
     } else if (warp == kRopeWarp) {
       // ---------- S-CTA rope producer: dims 512..575 of a tile's 128 rows, 32 TMA gathers of 4 rows ----------
       // (the TMA engine runs beside the cp.async path and adds to the gather rate of this SM)
       bool ok = true;
+      int issued = 0;  // tiles whose gathers went out
       if (lane == 0 && ntiles > 0) tma_prefetch_desc(&kvmap);
       for (int i = 0; i < ntiles && ok; ++i) {
         const int rs = i % kRSlots;
@@ -373,11 +380,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int32_t* rr = rows + i * kTile + 4 * lane;
         tma_gather4(base + Smem::kRRing + rs * kBlk + lane * 512, &kvmap, 512, max(rr[0], 0), max(rr[1], 0),
                     max(rr[2], 0), max(rr[3], 0), &bar[B_RFULL + rs]);
+        issued = i + 1;
       }
-      // no gather may still be landing when the CTA exits (the MMA normally consumed them all)
-      if (lane == 0 && ok)
-        for (int i = max(0, ntiles - kRSlots); i < ntiles; ++i)
-          mbar_wait(&bar[B_RFULL + i % kRSlots], (i / kRSlots) & 1, p.status, kDevErrTimeout);
+      // no gather may still be landing when the CTA exits, also after an error (the MMA normally
+      // consumed them all)
+      if (lane == 0)
+        for (int i = max(0, issued - kRSlots); i < issued; ++i)
+          mbar_drain(&bar[B_RFULL + i % kRSlots], (i / kRSlots) & 1, p.status);
       __syncwarp();
     } else {
       // ---------- S-CTA softmax (warps 21..28: thread = head h, keys 64*sub .. 64*sub+63) ----------
@@ -571,6 +580,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (i == ntiles - 1) mma_commit(&bar[B_OFINAL]);
           mma_commit_multicast(&bar[B_PFREE + pb], 1);  // to the S-CTA (rank 0)
         }
+        // every MMA this thread issued has completed before TMEM is freed (also after an error)
+        mma_commit(&bar[B_MDONE]);
+        mbar_drain(&bar[B_MDONE], 0, p.status);
       }
       __syncwarp();
     } else if (warp < kSoftWarp0 + kSoftWarps) {
@@ -673,6 +685,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
     }
   }
+  // the Q boxes may still be landing if an error ended the pipeline before Q was consumed
+  if (threadIdx.x == 0 && is_s && ntiles > 0) mbar_drain(&bar[B_QROPE], 0, p.status);
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();  // neither CTA leaves while the peer may still touch its shared memory
@@ -734,8 +748,8 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const float* __restric
 int sparse_mla_splits(int T, int k) {
   const int min_splits = (k + kMaxKeysPerCta - 1) / kMaxKeysPerCta;
   const int clusters_per_wave = 74;  // 148 SMs, two per cluster
-  int n = 1;
-  if (T > 0 && T < (3 * clusters_per_wave) / 4) n = (clusters_per_wave + T - 1) / T;
+  int n = 1;  // as many splits as keep every cluster of the launch in one wave
+  if (T > 0 && T < clusters_per_wave) n = clusters_per_wave / T;
   const int max_by_tiles = (k + kTile - 1) / kTile;
   if (n > 16) n = 16;
   if (n > max_by_tiles) n = max_by_tiles;

@@ -3,7 +3,10 @@
 // formula; when the prefix holds no more than k positions all of them are taken, the handbook's
 // k = min(L, TOPK) in "MTP 与稀疏注意力：NSA 与 DSA", section "稀疏注意力：NSA 与 DSA").
 //
-// One CTA of 1024 threads per query row; L = p + 1 visible scores.
+// Two kernels share the steps below. Batches of many rows (prefill) run one CTA of 1024 threads
+// per row. Batches of few rows (decode) would leave most SMs idle that way and pay one CTA's
+// latency chain per row, so there one cluster of up to 8 CTAs takes each row (topk_cluster_kernel,
+// further down). L = p + 1 visible scores.
 //  1. Scores become order-preserving uint32 keys (one float4 per thread per chunk of 4096
 //     positions, four chunks in flight); the row's smallest and largest key bound the search.
 //  2. A 2048-bin histogram linear in the score value between the row's minimum and maximum
@@ -30,6 +33,7 @@
 
 #include "dsa_internal.h"
 #include "dsa_ptx.cuh"
+#include "select_cluster.cuh"
 
 namespace dsa {
 namespace {
@@ -49,15 +53,17 @@ constexpr int kBinsPerThread = kBins / kThreads;  // descending bins owned by on
 static_assert(kBins % kThreads == 0 && kWarps <= 32, "bin ownership");
 
 __device__ __forceinline__ uint32_t order_key(float f) {
+  if (f != f) return 0u;  // NaN ranks below every other score, -inf included
   uint32_t b = __float_as_uint(f);
   if (b == 0x80000000u) b = 0u;  // -0 ranks as +0
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
-__device__ __forceinline__ float key_value(uint32_t u) {  // inverse of order_key (-0 comes back as +0)
+__device__ __forceinline__ float key_value(uint32_t u) {  // inverse of order_key (-0 -> +0, NaN -> a NaN)
   return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
 }
 
-// Block-wide inclusive scan of one value per thread; `scratch` holds kWarps ints.
+// Block-wide inclusive scan of one value per thread over NW warps; `scratch` holds NW ints.
+template <int NW = kWarps>
 __device__ __forceinline__ int block_inclusive_scan(int v, int* scratch, int* total) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   int x = v;
@@ -69,17 +75,17 @@ __device__ __forceinline__ int block_inclusive_scan(int v, int* scratch, int* to
   if (lane == 31) scratch[wid] = x;
   __syncthreads();
   if (wid == 0) {
-    int s = lane < kWarps ? scratch[lane] : 0;
+    int s = lane < NW ? scratch[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, s, o);
       if (lane >= o) s += y;
     }
-    if (lane < kWarps) scratch[lane] = s;
+    if (lane < NW) scratch[lane] = s;
   }
   __syncthreads();
   const int r = x + (wid > 0 ? scratch[wid - 1] : 0);
-  *total = scratch[kWarps - 1];
+  *total = scratch[NW - 1];
   __syncthreads();
   return r;
 }
@@ -90,9 +96,10 @@ struct Keys4 {
 
 // kMerge = false (slice mode): CTA (t, s) of a T x nsl_max grid selects among positions
 //   [s*kSlice, min(L, (s+1)*kSlice)) of row t. A row of one slice writes S_t itself; otherwise the
-//   slice's k winners (increasing positions, -1 padded) go to block (t, s) of the candidate space.
-// kMerge = true: CTA t selects among the candidates of row t (their scores gathered from the row),
-//   in candidate order = increasing position; rows of one slice have nothing to do here.
+//   slice's k winners (increasing positions, -1 padded) go to block (t, s) of the candidate space,
+//   and their keys to the same block of the key space that follows it.
+// kMerge = true: CTA t selects among the candidates of row t (keys read from the key space), in
+//   candidate order = increasing position; rows of one slice have nothing to do here.
 template <bool kMerge>
 __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restrict__ row_pos,
                                                         const float* __restrict__ scores, int64_t ld, int k,
@@ -118,14 +125,21 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
   const int base = sl * kSlice;
   // the n elements this CTA selects from: positions base + i, or the candidates of row t
   const int n = kMerge ? (nsl - 1) * k + min(k, L - (nsl - 1) * kSlice) : min(kSlice, L - base);
+  // candidate space: positions [T][nsl_max][kpad], then their keys in the same layout
+  const int64_t key_off = static_cast<int64_t>(gridDim.x / (kMerge ? 1 : nsl_max)) * nsl_max * kpad;
   const int32_t* cands = cand_ws + static_cast<int64_t>(t) * nsl_max * kpad;
+  const uint32_t* cand_keys = reinterpret_cast<const uint32_t*>(cands + key_off);
   auto position = [&](int i) -> int { return kMerge ? __ldg(cands + (i / k) * kpad + i % k) : base + i; };
-  int32_t* out = (kMerge || nsl == 1) ? S + static_cast<int64_t>(t) * k
-                                      : cand_ws + (static_cast<int64_t>(t) * nsl_max + sl) * kpad;
+  const bool to_cands = !kMerge && nsl > 1;
+  int32_t* out = to_cands ? cand_ws + (static_cast<int64_t>(t) * nsl_max + sl) * kpad : S + static_cast<int64_t>(t) * k;
+  uint32_t* out_key = to_cands ? reinterpret_cast<uint32_t*>(out + key_off) : nullptr;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
 
   if (n <= k) {
-    for (int j = tid; j < k; j += kThreads) out[j] = (j < n) ? position(j) : -1;
+    for (int j = tid; j < k; j += kThreads) {
+      out[j] = (j < n) ? position(j) : -1;
+      if (out_key) out_key[j] = (j < n) ? order_key(__ldg(row + base + j)) : 0u;
+    }
     return;
   }
   const int nchunks = (n + kChunk - 1) / kChunk;
@@ -156,11 +170,12 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
       const int j0 = (cg + g) * kChunk + 4 * tid;
       nv[g] = max(0, min(4, n - j0));
       if (nv[g] > 0) {
-        if (kMerge) {  // gather the candidates' scores
-          f[g].x = __ldg(row + position(j0));
-          f[g].y = nv[g] > 1 ? __ldg(row + position(j0 + 1)) : 0.f;
-          f[g].z = nv[g] > 2 ? __ldg(row + position(j0 + 2)) : 0.f;
-          f[g].w = nv[g] > 3 ? __ldg(row + position(j0 + 3)) : 0.f;
+        if (kMerge) {  // the candidates' keys, as the slice CTAs wrote them
+          float v[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (e < nv[g]) v[e] = key_value(__ldg(cand_keys + ((j0 + e) / k) * kpad + (j0 + e) % k));
+          f[g] = make_float4(v[0], v[1], v[2], v[3]);
         } else {  // base + j0 + 3 < ld: base and j0 are multiples of 4, ld % 4 == 0, base + j0 < L <= ld
           f[g] = __ldg(reinterpret_cast<const float4*>(row + base + j0));
         }
@@ -431,10 +446,15 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
         if (e >= nv[g]) break;
         const uint32_t u = r[g].k[e];
         if (u > theta) {
-          out[gt_before + min(eq_before, ties)] = position(j0 + e);
+          const int at = gt_before + min(eq_before, ties);
+          out[at] = position(j0 + e);
+          if (out_key) out_key[at] = u;
           ++gt_before;
         } else if (u == theta) {
-          if (eq_before < ties) out[gt_before + eq_before] = position(j0 + e);
+          if (eq_before < ties) {
+            out[gt_before + eq_before] = position(j0 + e);
+            if (out_key) out_key[gt_before + eq_before] = u;
+          }
           ++eq_before;
         }
       }
@@ -442,12 +462,91 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
   }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Cluster top-k for batches of few rows (decode): one cluster of C CTAs (C = 1, 2, 4 or 8) per row,
+// so that one row's latency chain is spread over C SMs. CTA r loads the scores of positions
+// [r*s, min(L, (r+1)*s)) into its shared memory as order-preserving keys, s = ceil(L/C) rounded up
+// to a multiple of 4; the selection over the whole row then runs in sel::select_topk, which
+// exchanges what it combines across the row through distributed shared memory.
+
+constexpr int kCThreads = 512;
+constexpr int kCChunk = 4 * kCThreads;             // positions per chunk (one float4 per thread)
+constexpr int kCMaxSlice = 16384;                  // positions per CTA
+constexpr int kCMaxCluster = sel::kMaxCluster;     // 8
+constexpr int kCMaxRow = kCMaxSlice * kCMaxCluster;  // 131072
+static_assert(kCMaxSlice <= kCChunk * sel::kMaxChunks && kBins == sel::kBins, "cluster top-k");
+
+__global__ void __launch_bounds__(kCThreads) topk_cluster_kernel(const int32_t* __restrict__ row_pos,
+                                                                 const float* __restrict__ scores, int64_t ld,
+                                                                 int k, int32_t* __restrict__ S, int slice_cap) {
+  extern __shared__ __align__(16) uint32_t tc_smem[];
+  __shared__ sel::Shared<kCThreads> sh;
+  const uint32_t C = cluster_nctarank(), rank = cluster_ctarank();
+  uint32_t* cache = tc_smem;             // [slice_cap] keys of this CTA's positions
+  uint32_t* hist = tc_smem + slice_cap;  // [sel::hist_words(C)]
+  const int t = static_cast<int>(blockIdx.x / C);
+  const int tid = threadIdx.x;
+
+  sel::clear_state<kCThreads>(sh, hist, C);
+  sel::cluster_arrive();  // waited for at the start of the selection (or before an early exit)
+  pdl_trigger();
+  pdl_wait();  // scores and plan from the previous kernels
+  const int L = __ldg(row_pos + t) + 1;
+  int32_t* out = S + static_cast<int64_t>(t) * k;
+  if (L <= k) {  // every visible position, then padding (the same branch in every CTA of the row)
+    const int per = (k + static_cast<int>(C) - 1) / static_cast<int>(C);
+    const int j1 = min(k, static_cast<int>(rank + 1) * per);
+    for (int j = static_cast<int>(rank) * per + tid; j < j1; j += kCThreads) out[j] = j < L ? j : -1;
+    sel::cluster_wait();
+    return;
+  }
+  const int s = ((L + static_cast<int>(C) - 1) / static_cast<int>(C) + 3) & ~3;
+  const int base = static_cast<int>(rank) * s;
+  const int n = max(0, min(L - base, s));
+  const float* row = scores + static_cast<int64_t>(t) * ld + base;
+  const int nchunks = (n + kCChunk - 1) / kCChunk;
+  for (int cg = 0; cg < nchunks; cg += kLoadGroup) {
+    float4 f[kLoadGroup];
+    int nv[kLoadGroup];
+#pragma unroll
+    for (int g = 0; g < kLoadGroup; ++g) {
+      const int j0 = (cg + g) * kCChunk + 4 * tid;
+      nv[g] = max(0, min(4, n - j0));
+      // base + j0 + 3 < ld: base and j0 are multiples of 4, ld % 4 == 0, base + j0 < L <= ld
+      if (nv[g] > 0) f[g] = __ldg(reinterpret_cast<const float4*>(row + j0));
+    }
+#pragma unroll
+    for (int g = 0; g < kLoadGroup; ++g) {
+      if (nv[g] == 0) continue;
+      *reinterpret_cast<uint4*>(cache + (cg + g) * kCChunk + 4 * tid) =
+          make_uint4(sel::order_key(f[g].x), sel::order_key(f[g].y), sel::order_key(f[g].z), sel::order_key(f[g].w));
+    }
+  }
+  __syncthreads();
+  sel::select_topk<kCThreads>(cache, n, base, k, out, sh, hist, C, rank);
+  sel::cluster_wait();  // no CTA leaves while a peer may still address its shared memory
+}
+
 }  // namespace
 
+// Cluster size of the cluster kernel for this batch, or 0 for the single-CTA kernel. Measured on
+// B200: for rows that fit one CTA (<= kSlice positions) the cluster's exchanges cost about what
+// splitting the row saves, so one CTA per row it is; rows above kSlice need the single-CTA kernel's
+// slices and a merge launch, which the cluster kernel avoids when all its clusters fit in one wave
+// (two CTAs per SM).
+int topk_cluster_size(int T, int max_seq_len) {
+  constexpr int kOneWave = 2 * 148;
+  if (max_seq_len <= kSlice || max_seq_len > kCMaxRow) return 0;
+  int c = 1;
+  while (c < kCMaxCluster && (max_seq_len + c - 1) / c > kCMaxSlice) c <<= 1;
+  return (T * c <= kOneWave) ? c : 0;
+}
+
 size_t topk_ws_bytes(int T, int max_seq_len, int k) {
+  if (topk_cluster_size(T, max_seq_len) > 0) return 0;
   const int nsl = (max_seq_len + kSlice - 1) / kSlice;
-  if (nsl <= 1) return 0;
-  return sizeof(int32_t) * static_cast<size_t>(T) * static_cast<size_t>(nsl) * static_cast<size_t>((k + 3) & ~3);
+  if (nsl <= 1) return 0;  // positions and keys of every slice's winners
+  return 2 * sizeof(int32_t) * static_cast<size_t>(T) * static_cast<size_t>(nsl) * static_cast<size_t>((k + 3) & ~3);
 }
 
 int launch_topk(const BatchDev& b, const void* plan, const float* scores, int64_t ld, int k, int32_t* S, void* ws,
@@ -455,6 +554,16 @@ int launch_topk(const BatchDev& b, const void* plan, const float* scores, int64_
   if (b.T == 0) return 0;
   if (b.max_seq_len > kMaxTopKRow) return static_cast<int>(cudaErrorInvalidValue);
   PlanView pv = plan_view(const_cast<void*>(plan), b.B, b.T);
+  const int C = topk_cluster_size(b.T, b.max_seq_len);
+  if (C > 0) {
+    const int slice_cap = ((b.max_seq_len + C - 1) / C + 3) & ~3;
+    const size_t smem = sizeof(uint32_t) * (static_cast<size_t>(slice_cap) + sel::hist_words(C));
+    cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return static_cast<int>(e);
+    return static_cast<int>(launch_pdl_cluster(topk_cluster_kernel, dim3(b.T * C), dim3(kCThreads), smem, stream,
+                                               static_cast<unsigned>(C), pv.row_pos, scores, ld, k, S, slice_cap));
+  }
   const int nsl = b.max_seq_len > kSlice ? (b.max_seq_len + kSlice - 1) / kSlice : 1;
   const int kpad = (k + 3) & ~3;
   if (nsl > 1 && !ws) return static_cast<int>(cudaErrorInvalidValue);

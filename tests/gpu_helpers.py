@@ -2,9 +2,9 @@
 the CPU oracle on the same seeded inputs.
 
 Tolerances (written out here, derived in the design notes):
-  * scores: |I_gpu - I_oracle| <= 1e-3 * |I_oracle| + 1e-3 * rms_t, rms_t = the RMS of row t's
-    oracle scores (FP8 products are exact; the error is fp32 accumulation and summation order, so
-    it scales with the magnitudes summed, not with the possibly cancelled result).
+  * scores: |I_gpu - I_oracle| <= 1e-3 * |I_oracle| + 1e-6 * max_j |I_oracle,tj| (the relative
+    1e-3 asked for, with a floor for scores near 0, where signed head weights can cancel: FP8
+    products are exact in fp32, the error is fp32 accumulation and summation order).
   * index sets: equal, except that every position in the symmetric difference has an oracle
     score within 1e-3 * |I_(k)| of the k-th largest oracle score I_(k) (near-ties).
   * top-k alone, fed the GPU's own fp32 scores: identical sets (both break ties by position).
@@ -48,9 +48,8 @@ def check_scores(ref: dict, got: dict, pos) -> float:
     worst = 0.0
     for t, r in ref.items():
         g = got[t][: pos[t] + 1].astype(np.float64)
-        rms = float(np.sqrt(np.mean(r * r)))
         err = np.abs(g - r)
-        bound = 1e-3 * np.abs(r) + 1e-3 * rms
+        bound = 1e-3 * np.abs(r) + 1e-6 * float(np.max(np.abs(r)))
         ratio = float(np.max(err / np.maximum(bound, 1e-30)))
         worst = max(worst, ratio)
         assert ratio <= 1.0, f"row {t}: score error {err.max():.3e} exceeds the bound (ratio {ratio:.2f})"

@@ -38,8 +38,8 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_strings(lib):
-    assert lib.dsa_abi_version() == 3
-    for s in range(7):
+    assert lib.dsa_abi_version() == 4
+    for s in range(8):
         assert lib.dsa_status_string(s).decode() == dsa.STATUS[s]
     assert lib.dsa_status_string(99).decode() == "unknown status"
 
@@ -119,11 +119,17 @@ def test_topk_and_mla_validation(lib):
     assert lib.dsa_topk(ctypes.byref(b), FAKE, FAKE + 4, 384, 16, FAKE, None, 0, None) == 1  # misaligned scores
     long_rows = batch(max_seq_len=262145, max_pages=4097)
     assert lib.dsa_topk(ctypes.byref(long_rows), FAKE, FAKE, 262148, 16, FAKE, None, 0, None) == 2
-    # rows above 32768 positions need the candidate workspace: T * slices * round4(k) int32
-    sliced = batch(max_seq_len=70000, max_pages=1094, num_pages=2000)
-    need = lib.dsa_topk_workspace_size(ctypes.byref(sliced), 2047)
-    assert need == 4 * 3 * 3 * 2048
+    # few rows of 32769 .. 131072 positions: one cluster of CTAs per row, no workspace
+    few = batch(max_seq_len=70000, max_pages=1094, num_pages=2000)
+    assert lib.dsa_topk_workspace_size(ctypes.byref(few), 2047) == 0
     assert lib.dsa_topk_workspace_size(ctypes.byref(b), 2048) == 0
+    # many long rows, or rows above 131072 positions: one CTA per row and 32768-position slice,
+    # whose winners wait in the candidate workspace: positions and keys, T * slices * round4(k) each
+    sliced = batch(B=1, T=1200, max_q=1200, max_seq_len=70000, max_pages=1094, num_pages=2000)
+    need = lib.dsa_topk_workspace_size(ctypes.byref(sliced), 2047)
+    assert need == 2 * 4 * 1200 * 3 * 2048
+    longest = batch(max_seq_len=140000, max_pages=2188, num_pages=3000)
+    assert lib.dsa_topk_workspace_size(ctypes.byref(longest), 2048) == 2 * 4 * 3 * 5 * 2048
     assert lib.dsa_topk(ctypes.byref(sliced), FAKE, FAKE, 70000, 2047, FAKE, None, 0, None) == 1      # no ws
     assert lib.dsa_topk(ctypes.byref(sliced), FAKE, FAKE, 70000, 2047, FAKE, FAKE, need - 1, None) == 3
     mla = lambda **kw: lib.dsa_sparse_mla(

@@ -37,19 +37,28 @@ def _new_rows(T, seed):
     return k_new, c_new
 
 
-def _run(wl, seed):
+def _run(wl, seed, bad_rows=()):
     hb = synth.make_batch(wl, seed=seed, extra_pages=3)
     db = dsa.DeviceBatch(hb)
     plan = dsa.plan(db.batch, db.nhI)
     T = hb.total_q
     k_new, c_new = _new_rows(T, seed + 100)
+    for i, t in enumerate(bad_rows):  # keys with no FP8 encoding: the row must not be written
+        k_new[t, 5 + i] = [np.inf, -np.inf, np.nan][i % 3]
     dsa.cache_write(db.batch, plan, torch.from_numpy(k_new).cuda(),
                     torch.from_numpy(c_new.view(np.int16)).cuda().view(torch.bfloat16),
                     db.kI_cache, db.kI_scale, db.kv_cache)
     torch.cuda.synchronize()
-    assert dsa.status_read(plan) == 0
-    want_kI, want_ks, want_kv = O.cache_write(hb.seq_lens, hb.cu_q, hb.block_table, k_new, c_new, hb.kI_cache,
+    assert dsa.status_read(plan) == (7 if bad_rows else 0)  # DSA_ERR_DEVICE_VALUE
+    good = [t for t in range(T) if t not in bad_rows]
+    k_ok = np.where(np.isfinite(k_new), k_new, 0.0).astype(np.float32)
+    want_kI, want_ks, want_kv = O.cache_write(hb.seq_lens, hb.cu_q, hb.block_table, k_ok, c_new, hb.kI_cache,
                                               hb.kI_scale, hb.kv_cache)
+    req, pos = O.query_positions(hb.seq_lens, hb.cu_q)
+    for t in bad_rows:  # the rejected rows keep the slots' old contents in all three caches
+        (pg,), (sl,) = O.physical_rows(hb.block_table[req[t]], [pos[t]])
+        want_kI[pg, sl], want_ks[pg, sl], want_kv[pg, sl] = hb.kI_cache[pg, sl], hb.kI_scale[pg, sl], hb.kv_cache[pg, sl]
+    assert len(good) + len(bad_rows) == T
     got_kI = db.kI_cache.view(torch.uint8).cpu().numpy()
     got_ks = db.kI_scale.cpu().numpy()
     got_kv = db.kv_cache.view(torch.int16).cpu().numpy().view(np.uint16)
@@ -66,3 +75,8 @@ def test_cache_write_ragged_small():
 
 def test_cache_write_decode_64x16k():
     _run(synth.workload("decode_64x16k"), seed=12)
+
+
+def test_cache_write_rejects_non_finite_keys():
+    wl = synth.custom("cache_write_bad", [300, 1000, 64, 2100], [2, 3, 1, 4], n_heads_index=64, topk=256, n_heads=16)
+    _run(wl, seed=13, bad_rows=(2, 5, 9))

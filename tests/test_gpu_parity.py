@@ -121,4 +121,4 @@ def test_workload_mixed_128():
 def test_workload_prefill_32k_sampled():
     T = 32768
     rows = sorted(set(list(range(0, T, 64)) + list(range(2040, 2057)) + list(range(T - 16, T))))
-    run_all_checks(synth.workload("prefill_32k"), rows=rows, check_layer=False)
+    run_all_checks(synth.workload("prefill_32k"), rows=rows)

@@ -520,3 +520,11 @@ def test_cost_model_matches_printed_table(golden_dir):
         assert round(rd[0] / rd[1], 1) == row["read_ratio"]
         assert [round(x / 1e12, 1) for x in pre] == row["prefill_tflops"]
         assert round(pre[0] / pre[1], 1) == row["prefill_ratio"]
+
+
+def test_topk_nan_scores_rank_below_everything():
+    """The pages leave NaN scores undefined; the library's reading: a NaN score ranks below every
+    other score, -inf included, and NaNs tie (the smaller position first)."""
+    s = np.array([1.0, np.nan, -np.inf, 2.0, np.nan, 0.0, -0.0])
+    assert O.topk_select(s, 7).tolist() == [3, 0, 5, 6, 2, 1, 4]
+    assert sorted(O.topk_select(s, 4).tolist()) == [0, 3, 5, 6]
