@@ -76,7 +76,7 @@ struct Shared {
   uint32_t cand_count;              // rank 0: candidates pushed so far
   uint32_t cand_key[kCandCap];      // rank 0: the candidates
   uint32_t cand_rank[kCandCap];     //   and the rank that holds each
-  uint32_t lkey[kCandCap];          // this CTA's copy of the candidates
+  alignas(16) uint32_t lkey[kCandCap];  // this CTA's copy of the candidates (read 16 bytes at a time)
   uint32_t lrank[kCandCap];
   uint32_t rgt[kMaxCluster], req[kMaxCluster];  // candidates above / equal to theta per rank
   uint32_t lo, remaining, ncand, slot, w0;
@@ -211,23 +211,16 @@ __device__ void select_topk(const uint32_t* keys, int n, int base, int k, int32_
   bool found = false, via_cands = false;
   int pass = 0;
 
-  auto histogram = [&](auto bin_of) {  // local hist[bin(key)] += 1 for bin(key) < kBins
+  // local hist[bin(key)] += 1 for bin(key) < kBins: one shared-memory atomic per key, no warp-wide
+  // steps (their latency per key costs more than the rare collisions of random bins)
+  auto histogram = [&](auto bin_of) {
     for (int c = 0; c < nchunks; ++c) {
       uint32_t r[4];
       const int nv = load4(c, r);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const uint32_t bin = e < nv ? bin_of(r[e]) : 0xffffffffu;
-        const bool in = bin < static_cast<uint32_t>(kBins);
-        const uint32_t act = __ballot_sync(0xffffffffu, in);
-        if (act == 0u) continue;
-        const int first = __ffs(act) - 1;
-        const uint32_t b0 = __shfl_sync(0xffffffffu, bin, first);
-        if (__all_sync(0xffffffffu, !in || bin == b0)) {
-          if (lane == first) atomicAdd(&hist[b0], static_cast<uint32_t>(__popc(act)));
-        } else if (in) {
-          atomicAdd(&hist[bin], 1u);
-        }
+        if (bin < static_cast<uint32_t>(kBins)) atomicAdd(&hist[bin], 1u);
       }
     }
     __syncthreads();
@@ -299,6 +292,10 @@ __device__ void select_topk(const uint32_t* keys, int n, int base, int k, int32_
       for (int c = 0; c < nchunks; ++c) {
         uint32_t r[4];
         const int nv = load4(c, r);
+        bool any = false;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) any |= e < nv && is_cand(r[e]);
+        if (!__any_sync(0xffffffffu, any)) continue;  // the common case: no candidate in this chunk
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const bool in = e < nv && is_cand(r[e]);
@@ -322,12 +319,18 @@ __device__ void select_topk(const uint32_t* keys, int n, int base, int k, int32_
     }
     if (tid < kMaxCluster) sh.rgt[tid] = 0u, sh.req[tid] = 0u;
     __syncthreads();
+    if (static_cast<uint32_t>(tid) >= ncand && tid < ((ncand + 3) & ~3u)) sh.lkey[tid] = 0u;  // padding
+    __syncthreads();
     uint32_t best = 0u;
     bool have = false;
     if (static_cast<uint32_t>(tid) < ncand) {
       const uint32_t v = sh.lkey[tid];
       uint32_t ge = 0;
-      for (uint32_t j = 0; j < ncand; ++j) ge += (sh.lkey[j] >= v) ? 1u : 0u;
+      for (uint32_t j = 0; j < ncand; j += 4) {  // 16-byte broadcast loads, four compares each
+        const uint4 w = *reinterpret_cast<const uint4*>(&sh.lkey[j]);
+        ge += (w.x >= v ? 1u : 0u) + (w.y >= v ? 1u : 0u) + (w.z >= v ? 1u : 0u) + (w.w >= v ? 1u : 0u);
+      }
+      if (v == 0u) ge -= ((ncand + 3) & ~3u) - ncand;  // the zero padding counted as >= 0
       if (ge >= remaining) best = v, have = true;
     }
     best = __reduce_max_sync(0xffffffffu, have ? best : 0u);
@@ -456,20 +459,16 @@ __device__ void select_topk(const uint32_t* keys, int n, int base, int k, int32_
     if (lane == 0) sh.cnt[c][wid] = make_int2(gt, eq);
   }
   __syncthreads();
-  if (wid == 0) {  // exclusive prefix over (chunk, warp) in position order
-    int2 carry = make_int2(static_cast<int>(gt0), static_cast<int>(eq0));
-    for (int c = 0; c < nchunks; ++c) {
-      const int2 v = lane < NT / 32 ? sh.cnt[c][lane] : make_int2(0, 0);
-      int2 x = v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int yx = __shfl_up_sync(0xffffffffu, x.x, o), yy = __shfl_up_sync(0xffffffffu, x.y, o);
-        if (lane >= o) x.x += yx, x.y += yy;
-      }
-      if (lane < NT / 32) sh.cnt[c][lane] = make_int2(carry.x + x.x - v.x, carry.y + x.y - v.y);
-      carry.x += __shfl_sync(0xffffffffu, x.x, 31);
-      carry.y += __shfl_sync(0xffffffffu, x.y, 31);
-    }
+  {  // exclusive prefix over (chunk, warp) in position order: one block scan, entry tid = (chunk, warp)
+    static_assert(kMaxChunks * (NT / 32) <= NT, "one (chunk, warp) entry per thread");
+    const int c = tid / (NT / 32), w = tid % (NT / 32);
+    const int2 v = c < nchunks ? sh.cnt[c][w] : make_int2(0, 0);
+    const int packed = (v.y << 16) | v.x;  // a CTA holds fewer than 65536 keys
+    int total;
+    const int incl = block_scan<NT>(packed, sh.scan_scratch, &total);
+    const uint32_t ex = static_cast<uint32_t>(incl - packed);  // the two 16-bit halves, unsigned
+    if (c < nchunks)
+      sh.cnt[c][w] = make_int2(static_cast<int>(gt0 + (ex & 0xffffu)), static_cast<int>(eq0 + (ex >> 16)));
   }
   __syncthreads();
   const int ties = static_cast<int>(remaining);

@@ -207,12 +207,18 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
   // theta = the largest candidate value v with #(candidates >= v) >= remaining; on return
   // `remaining` counts the keys equal to theta that are taken. cand[0 .. ncand) holds the keys.
   auto resolve_candidates = [&](uint32_t ncand) {
+    if (static_cast<uint32_t>(tid) >= ncand && tid < ((ncand + 3) & ~3u)) cand[tid] = 0u;  // padding
+    __syncthreads();
     uint32_t best = 0u;
     bool have = false;
     if (static_cast<uint32_t>(tid) < ncand) {
       const uint32_t v = cand[tid];
       uint32_t ge = 0;
-      for (uint32_t j = 0; j < ncand; ++j) ge += (cand[j] >= v) ? 1u : 0u;
+      for (uint32_t j = 0; j < ncand; j += 4) {  // 16-byte broadcast loads, four compares each
+        const uint4 w = *reinterpret_cast<const uint4*>(&cand[j]);
+        ge += (w.x >= v ? 1u : 0u) + (w.y >= v ? 1u : 0u) + (w.z >= v ? 1u : 0u) + (w.w >= v ? 1u : 0u);
+      }
+      if (v == 0u) ge -= ((ncand + 3) & ~3u) - ncand;  // the zero padding counted as >= 0
       if (ge >= remaining) best = v, have = true;
     }
     best = __reduce_max_sync(0xffffffffu, have ? best : 0u);
@@ -231,6 +237,10 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
       load_group(cg, r, nv);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
+        bool any = false;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) any |= e < nv[g] && pred(r[g].k[e]);
+        if (!__any_sync(0xffffffffu, any)) continue;  // the common case: no candidate in this chunk
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const bool in = e < nv[g] && pred(r[g].k[e]);
@@ -246,7 +256,8 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
     }
     __syncthreads();
   };
-  // hist[bin(key)] += 1 over the keys with bin(key) < kBins (one atomic per warp when all agree)
+  // hist[bin(key)] += 1 over the keys with bin(key) < kBins: one shared-memory atomic per key, no
+  // warp-wide steps (their latency per key costs more than the rare collisions of random bins)
   auto histogram = [&](auto bin_of) {
     for (int cg = 0; cg < nchunks; cg += G) {
       Keys4 r[G];
@@ -257,16 +268,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const uint32_t bin = e < nv[g] ? bin_of(r[g].k[e]) : 0xffffffffu;
-          const bool in = bin < static_cast<uint32_t>(kBins);
-          const uint32_t act = __ballot_sync(0xffffffffu, in);
-          if (act == 0u) continue;
-          const int first = __ffs(act) - 1;
-          const uint32_t b0 = __shfl_sync(0xffffffffu, bin, first);
-          if (__all_sync(0xffffffffu, !in || bin == b0)) {
-            if (lane == first) atomicAdd(&hist[b0], static_cast<uint32_t>(__popc(act)));
-          } else if (in) {
-            atomicAdd(&hist[bin], 1u);
-          }
+          if (bin < static_cast<uint32_t>(kBins)) atomicAdd(&hist[bin], 1u);
         }
       }
     }
@@ -397,20 +399,15 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
     }
   }
   __syncthreads();
-  if (wid == 0) {  // exclusive prefix over (chunk, warp) in position order
-    int2 carry = make_int2(0, 0);
-    for (int c = 0; c < nchunks; ++c) {
-      const int2 v = lane < kWarps ? cnt[c][lane] : make_int2(0, 0);
-      int2 x = v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int yx = __shfl_up_sync(0xffffffffu, x.x, o), yy = __shfl_up_sync(0xffffffffu, x.y, o);
-        if (lane >= o) x.x += yx, x.y += yy;
-      }
-      if (lane < kWarps) cnt[c][lane] = make_int2(carry.x + x.x - v.x, carry.y + x.y - v.y);
-      carry.x += __shfl_sync(0xffffffffu, x.x, 31);
-      carry.y += __shfl_sync(0xffffffffu, x.y, 31);
-    }
+  {  // exclusive prefix over (chunk, warp) in position order: one block scan, entry tid = (chunk, warp)
+    static_assert(kMaxChunks * kWarps <= kThreads, "one (chunk, warp) entry per thread");
+    const int c = tid / kWarps, w = tid % kWarps;
+    const int2 v = c < nchunks ? cnt[c][w] : make_int2(0, 0);
+    const int packed = (v.y << 16) | v.x;  // a CTA holds fewer than 65536 keys
+    int total;
+    const int incl = block_inclusive_scan(packed, scan_scratch, &total);
+    const uint32_t ex = static_cast<uint32_t>(incl - packed);  // the two 16-bit halves, unsigned
+    if (c < nchunks) cnt[c][w] = make_int2(static_cast<int>(ex & 0xffffu), static_cast<int>(ex >> 16));
   }
   __syncthreads();
   const int ties = static_cast<int>(remaining);
