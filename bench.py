@@ -144,11 +144,14 @@ def algorithmic(hb):
             rows_per_req += min(int(hb.seq_lens[b]), int(sel[lo:hi].sum()))
     mla_bytes = rows_per_req * 576 * 2 + int(sel.sum()) * 4 + T * H * 576 * 2 + T * H * 512 * 2
     mla_flops = int(sel.sum()) * (2 * H * 576 + 2 * H * 512)
-    return dict(index_scores=(idx_bytes, idx_flops), topk=(topk_bytes, 0), sparse_mla=(mla_bytes, mla_flops))
+    # fused indexer + top-k: the keys, queries and weights, and the index sets written (no score rows)
+    fused_bytes = idx_bytes - int(vis.sum()) * 4 + T * k * 4
+    return dict(index_scores=(idx_bytes, idx_flops), topk=(topk_bytes, 0), sparse_mla=(mla_bytes, mla_flops),
+                index_topk=(fused_bytes, idx_flops))
 
 
 # the tensor dtype of each stage's contraction (the indexer is FP8, the sparse MLA bf16)
-STAGE_TENSOR = {"index_scores": "fp8", "topk": None, "sparse_mla": "bf16"}
+STAGE_TENSOR = {"index_scores": "fp8", "topk": None, "sparse_mla": "bf16", "index_topk": "fp8"}
 
 
 def stage_roofline(name: str, nbytes: int, flops: int, us: float, peaks: dict) -> dict:
@@ -374,6 +377,9 @@ class Runner:
         }
         self.layer = lambda: dsa.layer(db.batch, db.qI, db.qI_scale, db.wI, db.kI_cache, db.kI_scale, db.q,
                                        db.kv_cache, db.k, db.softmax_scale, out=self.out, ws=self.ws)
+        self.fused_ok = dsa.index_topk_supported(db.batch, db.nhI, db.k)
+        self.fused = lambda: dsa.index_topk(db.batch, self.plan, db.qI, db.qI_scale, db.wI, db.kI_cache,
+                                            db.kI_scale, db.k, S=self.S)
         self.replan = lambda: dsa.plan(db.batch, db.nhI, self.plan)
 
     def step(self):
@@ -431,6 +437,25 @@ def measure_workload(dsa, torch, wl, dev, seed, steps, warmup, flush, sampler, p
            "q_tok_s": hb.total_q / (ms / 1e3), "layer_with_plan_us": 1e3 * layer_ms, "plan_us": 1e3 * plan_ms,
            "layer_roofline_us": layer_roof_us, "layer_frac": layer_roof_us / (1e3 * ms),
            "launches_per_step": r.launches_per_step(), "stages": stages}
+    if r.fused_ok:
+        # the fused indexer + top-k (score rows never in memory) and the layer it makes with the sparse MLA
+        mla = r.stages["sparse_mla"]
+        fused_layer = lambda: (r.fused(), mla())
+        for _ in range(max(warmup, 0)):
+            fused_layer()
+        torch.cuda.synchronize()
+        if dsa.status_read(r.plan) != 0:
+            raise RuntimeError(f"{wl.name}: device status after the fused warm-up")
+        with sampler:
+            f_ms = timed_steps(torch, fused_layer, steps, flush, stream)
+        f_ms = max_over_ranks(f_ms, dist, dev)
+        fu_ms = timed_steps(torch, r.fused, n_extra, flush, stream)
+        st = stage_roofline("index_topk", work["index_topk"][0], work["index_topk"][1], 1e3 * fu_ms, peaks)
+        rep["fused"] = {"layer_us": 1e3 * f_ms, "q_tok_s": hb.total_q / (f_ms / 1e3), "index_topk": st,
+                        "saved_bytes_per_step": work["index_scores"][0] + work["topk"][0] - work["index_topk"][0],
+                        "launches_per_step": 2 + (1 if r.mla_ws_n > 0 else 0),
+                        "note": "dsa_index_topk + dsa_sparse_mla per step: no score rows in memory, one launch "
+                                "fewer than dsa_index_scores + dsa_topk"}
     if wl.name in DECODE_WORKLOADS or hb.total_q <= 256:
         # the benchmark spec's composite: the top-k and the gather/attention together against HBM
         tb = stages["topk"]["algorithmic_bytes"] + stages["sparse_mla"]["algorithmic_bytes"]

@@ -137,6 +137,25 @@ size_t dsa_topk_workspace_size(const dsa_batch_t* batch, int k);
 dsa_status_t dsa_topk(const dsa_batch_t* batch, const void* plan, const float* scores, int64_t ld, int k,
                       int32_t* S, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- steps 1 and 2 fused, for decode batches ---------------------------------------------
+ * The score rows never reach memory: one cluster of CTAs per request scores its keys into shared
+ * memory (the indexer's FP8 tcgen05 GEMM and epilogue) and selects there, the CTAs exchanging
+ * histograms, candidates and counts through distributed shared memory. ("MTP 与稀疏注意力：NSA 与
+ * DSA", section "对推理引擎的新要求": FP8 scoring and a per-query top-k over tens of thousands of
+ * positions are the kernels DSA asks of an engine; "DeepSeek Sparse Attention：从 SWA 到稀疏
+ * Attention 计算", Lightning Indexer section, formulas for I_tj and S_t.)
+ * Arguments as for dsa_index_scores and dsa_topk; S int32 [T, k] receives what dsa_topk writes for
+ * the scores dsa_index_scores computes (the same fp32 arithmetic: the same sets). The plan must be
+ * made for this batch (its status word records run-time faults). No workspace.
+ * Supported when every request's queries fit one indexer MMA group (max_q <= 256 / nhI) and a
+ * request's scores fit the shared memory of at most 8 CTAs (max_seq_len <= 131072 for one query
+ * per request, less for more); dsa_index_topk_supported returns 1 then (and for an empty batch),
+ * else 0, and dsa_index_topk returns DSA_ERR_UNSUPPORTED without launching. */
+int dsa_index_topk_supported(const dsa_batch_t* batch, int nhI, int k);
+dsa_status_t dsa_index_topk(const dsa_batch_t* batch, const void* plan, const uint8_t* qI, const float* qI_scale,
+                            const float* wI, int nhI, const uint8_t* kI_cache, const float* kI_scale, int k,
+                            int32_t* S, void* stream);
+
 /* ---- step 3: sparse MLA -----------------------------------------------------------------
  * q        bf16 [T, H, 576]     absorbed MLA queries, 1 <= H <= 128
  * kv_cache bf16 [P, 64, 576]    latent rows, paged

@@ -40,7 +40,7 @@ class DsaBatchC(ctypes.Structure):
 
 
 EXPORTS = ("dsa_abi_version", "dsa_status_string", "dsa_plan_workspace_size", "dsa_plan", "dsa_status_read",
-           "dsa_index_scores", "dsa_topk_workspace_size", "dsa_topk", "dsa_sparse_mla_workspace_size", "dsa_sparse_mla",
+           "dsa_index_scores", "dsa_index_topk_supported", "dsa_index_topk", "dsa_topk_workspace_size", "dsa_topk", "dsa_sparse_mla_workspace_size", "dsa_sparse_mla",
            "dsa_layer_workspace_size", "dsa_layer", "dsa_layer_noalloc", "dsa_layer_noalloc_status_read", "dsa_cache_write",
            "dsa_masked_mha_workspace_size", "dsa_masked_mha")
 
@@ -64,6 +64,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "dsa_plan": (I, [BP, I, P, SZ, P]),
         "dsa_status_read": (I, [P, P]),
         "dsa_index_scores": (I, [BP, P, P, P, P, I, P, P, P, I64, P]),
+        "dsa_index_topk_supported": (I, [BP, I, I]),
+        "dsa_index_topk": (I, [BP, P, P, P, P, I, P, P, I, P, P]),
         "dsa_topk_workspace_size": (SZ, [BP, I]),
         "dsa_topk": (I, [BP, P, P, I64, I, P, P, SZ, P]),
         "dsa_sparse_mla_workspace_size": (SZ, [BP, I, I]),
@@ -190,6 +192,28 @@ def index_scores(batch: Batch, plan_ws, qI, qI_scale, wI, kI_cache, kI_scale, sc
                                    wI.data_ptr(), nhI, kI_cache.data_ptr(), kI_scale.data_ptr(), scores.data_ptr(),
                                    ld, _stream()), "dsa_index_scores")
     return scores
+
+
+def index_topk_supported(batch: Batch, nhI: int, k: int) -> bool:
+    return bool(load().dsa_index_topk_supported(batch.ref(), nhI, k))
+
+
+def index_topk(batch: Batch, plan_ws, qI, qI_scale, wI, kI_cache, kI_scale, k: int, S=None) -> torch.Tensor:
+    """Indexer scores and top-k fused (dsa_index_topk): S [T, k] int32 without score rows in memory."""
+    T = batch.total_q
+    nhI = int(qI.shape[1])
+    _need(qI, "qI", torch.float8_e4m3fn, (T, nhI, D_INDEX))
+    _need(qI_scale, "qI_scale", torch.float32, (T,))
+    _need(wI, "wI", torch.float32, (T, nhI))
+    _need(kI_cache, "kI_cache", torch.float8_e4m3fn)
+    _need(kI_scale, "kI_scale", torch.float32)
+    if S is None:
+        S = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    _need(S, "S", torch.int32, (T, k))
+    _check(load().dsa_index_topk(batch.ref(), plan_ws.data_ptr(), qI.data_ptr(), qI_scale.data_ptr(), wI.data_ptr(),
+                                 nhI, kI_cache.data_ptr(), kI_scale.data_ptr(), k, S.data_ptr(), _stream()),
+           "dsa_index_topk")
+    return S
 
 
 def topk(batch: Batch, plan_ws, scores: torch.Tensor, k: int, S=None, ws=None) -> torch.Tensor:

@@ -137,6 +137,26 @@ dsa_status_t dsa_index_scores(const dsa_batch_t* batch, const void* plan, const 
                                        stream));
 }
 
+int dsa_index_topk_supported(const dsa_batch_t* batch, int nhI, int k) {
+  if (check_batch(batch) != DSA_OK || !valid_nhI(nhI) || k < 1 || k > kMaxTopK) return 0;
+  if (batch->total_q == 0) return 1;
+  return index_topk_cluster_size(batch->num_requests, batch->max_q, batch->max_seq_len, nhI) > 0 ? 1 : 0;
+}
+
+dsa_status_t dsa_index_topk(const dsa_batch_t* batch, const void* plan, const uint8_t* qI, const float* qI_scale,
+                            const float* wI, int nhI, const uint8_t* kI_cache, const float* kI_scale, int k,
+                            int32_t* S, void* stream) {
+  dsa_status_t st = check_batch(batch);
+  if (st != DSA_OK) return st;
+  if (!valid_nhI(nhI) || k < 1 || k > kMaxTopK) return DSA_ERR_UNSUPPORTED;
+  if (batch->total_q == 0) return DSA_OK;
+  if (!plan || !qI || !qI_scale || !wI || !kI_cache || !kI_scale || !S) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(plan) || !aligned16(qI) || !aligned16(kI_cache) || !aligned16(kI_scale) || !aligned16(wI))
+    return DSA_ERR_INVALID_ARG;
+  if (!dsa_index_topk_supported(batch, nhI, k)) return DSA_ERR_UNSUPPORTED;
+  return from_cuda(launch_index_topk(to_dev(batch), plan, qI, qI_scale, wI, nhI, kI_cache, kI_scale, k, S, stream));
+}
+
 size_t dsa_topk_workspace_size(const dsa_batch_t* batch, int k) {
   if (check_batch(batch) != DSA_OK || k < 1 || k > kMaxTopK || batch->max_seq_len > kMaxTopKRow) return 0;
   return topk_ws_bytes(batch->total_q, batch->max_seq_len, k);

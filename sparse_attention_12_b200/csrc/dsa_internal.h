@@ -114,6 +114,9 @@ int launch_cache_write(const BatchDev& b, const void* plan, const float* k_new, 
 int launch_index_scores(const BatchDev& b, const void* plan, const uint8_t* qI, const float* qI_scale,
                         const float* wI, int nhI, const uint8_t* kI_cache, const float* kI_scale, float* scores,
                         int64_t ld, void* stream);
+int index_topk_cluster_size(int B, int max_q, int max_seq_len, int nhI);
+int launch_index_topk(const BatchDev& b, const void* plan, const uint8_t* qI, const float* qI_scale, const float* wI,
+                      int nhI, const uint8_t* kI_cache, const float* kI_scale, int k, int32_t* S, void* stream);
 size_t topk_ws_bytes(int T, int max_seq_len, int k);
 int launch_topk(const BatchDev& b, const void* plan, const float* scores, int64_t ld, int k, int32_t* S, void* ws,
                 void* stream);

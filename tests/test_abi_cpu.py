@@ -216,3 +216,30 @@ def test_noalloc_checks_arguments_like_layer(lib):
     for bad in ({"qI": None}, {"out": None}, {"qI": FAKE + 4}, {"scale": 0.0}):
         assert noalloc(**bad) == layer(**bad) == 1, bad
     assert noalloc() == 3  # valid arguments, above the 64 MiB static array: DSA_ERR_WORKSPACE
+
+
+@no_gpu
+def test_index_topk_support_and_validation(lib):
+    def sup(B, T, max_q, L, nhI=64, k=2048):
+        b = dsa.DsaBatchC(B, T, max_q, L, (L + 63) // 64, B * ((L + 63) // 64), FAKE, FAKE, FAKE)
+        return lib.dsa_index_topk_supported(ctypes.byref(b), nhI, k)
+    assert sup(64, 64, 1, 16384) == 1          # decode: one query per request
+    assert sup(16, 32, 2, 131072) == 1         # MTP verify: two queries per request, long contexts
+    assert sup(128, 128, 1, 131072) == 1
+    assert sup(8, 32, 4, 32768) == 1           # four queries per request: one MMA group of 256 columns
+    assert sup(8, 32, 4, 65536) == 0           # ... whose scores of 8192 positions per CTA leave < 3 key stages
+    assert sup(8, 40, 5, 4096) == 0            # five do not fit one group of 64-head queries
+    assert sup(8, 128, 16, 4096, nhI=16) == 1  # sixteen 16-head queries do
+    assert sup(8, 32, 4, 131072) == 0          # four queries x 16384 positions per CTA: too much shared memory
+    assert sup(1, 4096, 4096, 4096) == 0       # a prefill: not one group
+    assert sup(64, 64, 1, 16384, nhI=48) == 0
+    b = dsa.DsaBatchC(2, 3, 2, 300, 5, 10, FAKE, FAKE, FAKE)
+    call = lambda **kw: lib.dsa_index_topk(ctypes.byref(kw.get("b", b)), FAKE, kw.get("qI", FAKE), FAKE, FAKE,
+                                           kw.get("nhI", 64), FAKE, FAKE, kw.get("k", 256), kw.get("S", FAKE), None)
+    assert call(S=None) == 1
+    assert call(qI=FAKE + 4) == 1
+    assert call(nhI=20) == 2
+    assert call(k=0) == 2
+    assert call(b=dsa.DsaBatchC(2, 6, 5, 300, 5, 10, FAKE, FAKE, FAKE)) == 2  # five queries in one request
+    empty = dsa.DsaBatchC(0, 0, 0, 0, 0, 0, None, None, None)
+    assert lib.dsa_index_topk(ctypes.byref(empty), None, None, None, None, 64, None, None, 256, None, None) == 0

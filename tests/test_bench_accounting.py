@@ -41,8 +41,10 @@ def test_decode_64x16k_bytes_and_flops():
     assert w["sparse_mla"][0] == 64 * (gather + q_mla + out)
     assert w["sparse_mla"][1] == 64 * 2048 * (2 * 128 * 576 + 2 * 128 * 512)
     # the method's own traffic without the score and index round trips: 4.81 MB per request
-    total = sum(v[0] for v in w.values())
+    total = sum(w[n][0] for n in ("index_scores", "topk", "sparse_mla"))
     assert total - 64 * (2 * scores + 2 * 2048 * 4) == 64 * 4808964
+    # fused indexer + top-k: no score row written or read, the index sets written
+    assert w["index_topk"][0] == 64 * (keys + qw + 2048 * 4)
 
 
 def test_causal_prefill_counts_visible_positions_only():
