@@ -38,19 +38,14 @@
 namespace dsa {
 namespace {
 
-constexpr int kThreads = 1024;
-constexpr int kWarps = kThreads / 32;
+constexpr int kWarps = 32;            // warps of a 1024-thread CTA (the block scan's default)
 constexpr int kBins = 2048;
-constexpr int kChunk = 4 * kThreads;  // positions per chunk (one float4 per thread)
-constexpr int kSlice = 32768;         // positions per CTA: their keys sit in shared memory (128 KB)
+constexpr int kSlice = 32768;         // most positions per CTA: their keys sit in shared memory (128 KB)
+constexpr int kSliceMany = 16384;     // slice for batches of many rows (64 KB: three CTAs per SM)
 constexpr int kCandCap = 128;         // candidates resolved by counting
 constexpr int kLoadGroup = 4;         // chunks whose global loads are in flight together
-constexpr int kMaxChunks = kSlice / kChunk;  // 8 chunks of 4096 positions per CTA
-constexpr int kMaxSlices = kMaxTopKRow / kSlice;  // rows up to 262144 positions: 8 slices
-static_assert(kMaxChunks % kLoadGroup == 0 && kMaxSlices * kMaxTopK <= kSlice, "a merge fits one CTA");
-static_assert(kCandCap <= kThreads, "one candidate per thread");
-constexpr int kBinsPerThread = kBins / kThreads;  // descending bins owned by one thread in the scan
-static_assert(kBins % kThreads == 0 && kWarps <= 32, "bin ownership");
+constexpr int kMaxSlices = kMaxTopKRow / kSlice;  // rows up to 262144 positions: 8 slices of kSlice
+static_assert(kMaxSlices * kMaxTopK <= kSlice, "a merge of kSlice-position slices fits one CTA");
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   if (f != f) return 0u;  // NaN ranks below every other score, -inf included
@@ -100,15 +95,24 @@ struct Keys4 {
 //   and their keys to the same block of the key space that follows it.
 // kMerge = true: CTA t selects among the candidates of row t (keys read from the key space), in
 //   candidate order = increasing position; rows of one slice have nothing to do here.
-template <bool kMerge>
-__global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restrict__ row_pos,
-                                                        const float* __restrict__ scores, int64_t ld, int k,
-                                                        int32_t* __restrict__ S, int32_t* __restrict__ cand_ws,
-                                                        int nsl_max, int kpad) {
+// NT threads per CTA (1024 for batches of few rows: the shortest chain per row; 512 for batches of
+// many rows, whose 16384-position slices then leave room for three CTAs per SM). `slice`: positions
+// per slice CTA (kSlice or kSliceMany); a row of nsl slices has nsl * k <= kSlice candidates.
+template <bool kMerge, int NT>
+__global__ void __launch_bounds__(NT) topk_kernel(const int32_t* __restrict__ row_pos,
+                                                  const float* __restrict__ scores, int64_t ld, int k,
+                                                  int32_t* __restrict__ S, int32_t* __restrict__ cand_ws,
+                                                  int nsl_max, int kpad, int slice) {
+  constexpr int kThreads = NT;
+  constexpr int kWarps = NT / 32;
+  constexpr int kChunk = 4 * NT;                 // positions per chunk (one float4 per thread)
+  constexpr int kMaxChunks = kSlice / kChunk;    // 8 (NT = 1024) or 16 (NT = 512) chunks per CTA
+  constexpr int kBinsPerThread = kBins / NT;     // descending bins owned by one thread in the scan
+  static_assert(kMaxChunks % kLoadGroup == 0 && kCandCap <= NT && kBins % NT == 0 && kWarps <= 32, "top-k CTA");
   extern __shared__ __align__(16) uint32_t tk_smem[];
   uint32_t* hist = tk_smem;                 // [kBins]
   uint32_t* cand = tk_smem + kBins;         // [kCandCap]
-  uint32_t* cache = cand + kCandCap;        // [kSlice] keys of this CTA's positions
+  uint32_t* cache = cand + kCandCap;        // [slice] keys of this CTA's positions
   __shared__ int scan_scratch[kWarps];
   __shared__ uint32_t red_min[kWarps], red_max[kWarps];
   __shared__ uint32_t sh_lo, sh_remaining, sh_ncand, sh_done;
@@ -119,12 +123,12 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
   pdl_trigger();
   pdl_wait();  // scores, plan and candidates from the previous kernels
   const int L = __ldg(row_pos + t) + 1;
-  const int nsl = (L + kSlice - 1) / kSlice;
+  const int nsl = (L + slice - 1) / slice;
   if (kMerge ? nsl <= 1 : sl >= nsl) return;
   const float* row = scores + static_cast<int64_t>(t) * ld;
-  const int base = sl * kSlice;
+  const int base = sl * slice;
   // the n elements this CTA selects from: positions base + i, or the candidates of row t
-  const int n = kMerge ? (nsl - 1) * k + min(k, L - (nsl - 1) * kSlice) : min(kSlice, L - base);
+  const int n = kMerge ? (nsl - 1) * k + min(k, L - (nsl - 1) * slice) : min(slice, L - base);
   // candidate space: positions [T][nsl_max][kpad], then their keys in the same layout
   const int64_t key_off = static_cast<int64_t>(gridDim.x / (kMerge ? 1 : nsl_max)) * nsl_max * kpad;
   const int32_t* cands = cand_ws + static_cast<int64_t>(t) * nsl_max * kpad;
@@ -286,7 +290,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
       sum += cnts[q];
     }
     int total;
-    const int incl = block_inclusive_scan(static_cast<int>(sum), scan_scratch, &total);
+    const int incl = block_inclusive_scan<kWarps>(static_cast<int>(sum), scan_scratch, &total);
     uint32_t before = static_cast<uint32_t>(incl) - sum;
 #pragma unroll
     for (int q = 0; q < kBinsPerThread; ++q) {
@@ -405,7 +409,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const int32_t* __restric
     const int2 v = c < nchunks ? cnt[c][w] : make_int2(0, 0);
     const int packed = (v.y << 16) | v.x;  // a CTA holds fewer than 65536 keys
     int total;
-    const int incl = block_inclusive_scan(packed, scan_scratch, &total);
+    const int incl = block_inclusive_scan<kWarps>(packed, scan_scratch, &total);
     const uint32_t ex = static_cast<uint32_t>(incl - packed);  // the two 16-bit halves, unsigned
     if (c < nchunks) cnt[c][w] = make_int2(static_cast<int>(ex & 0xffffu), static_cast<int>(ex >> 16));
   }
@@ -539,12 +543,50 @@ int topk_cluster_size(int T, int max_seq_len) {
   return (T * c <= kOneWave) ? c : 0;
 }
 
+// Slice size of the single-CTA kernel: 16384 positions (512-thread CTAs, three per SM) for batches
+// of many rows, whose throughput is what counts, when the slices' winners still fit one merge CTA;
+// else 32768 (1024-thread CTAs: the shortest chain per row).
+namespace {
+constexpr int kManyRows = 8 * 148;
+int single_cta_slice(int T, int max_seq_len, int k) {
+  const int nsl = (max_seq_len + kSliceMany - 1) / kSliceMany;
+  return (T >= kManyRows && nsl * k <= kSlice) ? kSliceMany : kSlice;
+}
+}  // namespace
+
 size_t topk_ws_bytes(int T, int max_seq_len, int k) {
   if (topk_cluster_size(T, max_seq_len) > 0) return 0;
-  const int nsl = (max_seq_len + kSlice - 1) / kSlice;
+  const int slice = single_cta_slice(T, max_seq_len, k);
+  const int nsl = (max_seq_len + slice - 1) / slice;
   if (nsl <= 1) return 0;  // positions and keys of every slice's winners
   return 2 * sizeof(int32_t) * static_cast<size_t>(T) * static_cast<size_t>(nsl) * static_cast<size_t>((k + 3) & ~3);
 }
+
+namespace {
+template <int NT>
+int launch_topk_single(const BatchDev& b, const PlanView& pv, const float* scores, int64_t ld, int k, int32_t* S,
+                       void* ws, int slice, void* stream) {
+  const int nsl = (b.max_seq_len + slice - 1) / slice;
+  const int kpad = (k + 3) & ~3;
+  if (nsl > 1 && !ws) return static_cast<int>(cudaErrorInvalidValue);
+  int32_t* cand_ws = static_cast<int32_t*>(ws);
+  const int max_smem = static_cast<int>(sizeof(uint32_t) * (kBins + kCandCap + kSlice));
+  for (auto kern : {topk_kernel<false, NT>, topk_kernel<true, NT>}) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+    if (e != cudaSuccess) return static_cast<int>(e);
+  }
+  const int capA = std::min(slice, (b.max_seq_len + 3) & ~3);
+  cudaError_t e = launch_pdl(topk_kernel<false, NT>, dim3(b.T * nsl), dim3(NT),
+                             sizeof(uint32_t) * (kBins + kCandCap + static_cast<size_t>(capA)), stream, pv.row_pos,
+                             scores, ld, k, S, cand_ws, nsl, kpad, slice);
+  if (e != cudaSuccess || nsl == 1) return static_cast<int>(e);
+  const int capB = std::min(kSlice, (nsl * k + 3) & ~3);
+  e = launch_pdl(topk_kernel<true, NT>, dim3(b.T), dim3(NT),
+                 sizeof(uint32_t) * (kBins + kCandCap + static_cast<size_t>(capB)), stream, pv.row_pos, scores, ld, k,
+                 S, cand_ws, nsl, kpad, slice);
+  return static_cast<int>(e);
+}
+}  // namespace
 
 int launch_topk(const BatchDev& b, const void* plan, const float* scores, int64_t ld, int k, int32_t* S, void* ws,
                 void* stream) {
@@ -561,25 +603,9 @@ int launch_topk(const BatchDev& b, const void* plan, const float* scores, int64_
     return static_cast<int>(launch_pdl_cluster(topk_cluster_kernel, dim3(b.T * C), dim3(kCThreads), smem, stream,
                                                static_cast<unsigned>(C), pv.row_pos, scores, ld, k, S, slice_cap));
   }
-  const int nsl = b.max_seq_len > kSlice ? (b.max_seq_len + kSlice - 1) / kSlice : 1;
-  const int kpad = (k + 3) & ~3;
-  if (nsl > 1 && !ws) return static_cast<int>(cudaErrorInvalidValue);
-  int32_t* cand_ws = static_cast<int32_t*>(ws);
-  const int max_smem = static_cast<int>(sizeof(uint32_t) * (kBins + kCandCap + kSlice));
-  for (auto kern : {topk_kernel<false>, topk_kernel<true>}) {
-    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
-    if (e != cudaSuccess) return static_cast<int>(e);
-  }
-  const int capA = std::min(kSlice, (b.max_seq_len + 3) & ~3);
-  cudaError_t e = launch_pdl(topk_kernel<false>, dim3(b.T * nsl), dim3(kThreads),
-                             sizeof(uint32_t) * (kBins + kCandCap + static_cast<size_t>(capA)), stream, pv.row_pos,
-                             scores, ld, k, S, cand_ws, nsl, kpad);
-  if (e != cudaSuccess || nsl == 1) return static_cast<int>(e);
-  const int capB = std::min(kSlice, (nsl * k + 3) & ~3);
-  e = launch_pdl(topk_kernel<true>, dim3(b.T), dim3(kThreads),
-                 sizeof(uint32_t) * (kBins + kCandCap + static_cast<size_t>(capB)), stream, pv.row_pos, scores, ld, k,
-                 S, cand_ws, nsl, kpad);
-  return static_cast<int>(e);
+  const int slice = single_cta_slice(b.T, b.max_seq_len, k);
+  return slice == kSliceMany ? launch_topk_single<512>(b, pv, scores, ld, k, S, ws, slice, stream)
+                             : launch_topk_single<1024>(b, pv, scores, ld, k, S, ws, slice, stream);
 }
 
 }  // namespace dsa

@@ -88,6 +88,10 @@ def workload(name: str, seed: int = 0) -> Workload:
         rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, 5, 1])))
         lens = _log_uniform_lengths(rng, 128, 4096, 131072)
         return Workload(name, 5, lens, (1,) * 128, 64, 2048, 128, "none", 0)
+    if name.startswith("prefill_") and name[len("prefill_"):].isdigit():
+        # prefill_32k's shape at another length L (smaller cases of the same kernels, for profiling)
+        L = int(name[len("prefill_"):])
+        return Workload(name, 6, (L,), (L,), 64, 2048, 128, "prefill_logdist", max(1, L // 512))
     raise KeyError(name)
 
 

@@ -125,9 +125,13 @@ def test_topk_and_mla_validation(lib):
     assert lib.dsa_topk_workspace_size(ctypes.byref(b), 2048) == 0
     # many long rows, or rows above 131072 positions: one CTA per row and 32768-position slice,
     # whose winners wait in the candidate workspace: positions and keys, T * slices * round4(k) each
+    # (batches of many rows take 16384-position slices while the slices' winners fit one merge CTA)
     sliced = batch(B=1, T=1200, max_q=1200, max_seq_len=70000, max_pages=1094, num_pages=2000)
     need = lib.dsa_topk_workspace_size(ctypes.byref(sliced), 2047)
-    assert need == 2 * 4 * 1200 * 3 * 2048
+    assert need == 2 * 4 * 1200 * 5 * 2048
+    wide_k = batch(B=1, T=1200, max_q=1200, max_seq_len=140000, max_pages=2188, num_pages=3000)
+    # 9 slices of 16384 x 4096 winners > 32768: slices of 32768 instead
+    assert lib.dsa_topk_workspace_size(ctypes.byref(wide_k), 4096) == 2 * 4 * 1200 * 5 * 4096
     longest = batch(max_seq_len=140000, max_pages=2188, num_pages=3000)
     assert lib.dsa_topk_workspace_size(ctypes.byref(longest), 2048) == 2 * 4 * 3 * 5 * 2048
     assert lib.dsa_topk(ctypes.byref(sliced), FAKE, FAKE, 70000, 2047, FAKE, None, 0, None) == 1      # no ws

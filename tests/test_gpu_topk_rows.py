@@ -118,3 +118,11 @@ def test_topk_many_long_rows_slices_and_merge():
     kinds = ["normal", "three_values", "narrow", "wide", "zeros_inf", "flat"]
     rows = [(kinds[i % len(kinds)], 32769 + (i * 2467) % 98000) for i in range(40)]
     _run(2048, rows, seed=6)
+
+
+def test_topk_many_rows_with_long_ones_slices_of_16384():
+    # 1200 rows, every 97th of them 40000 positions long: 512-thread CTAs over 16384-position slices,
+    # a merge for the long rows
+    kinds = ["normal", "three_values", "narrow", "wide", "zeros_inf", "nans"]
+    rows = [(kinds[i % len(kinds)], 40000 if i % 97 == 0 else 300 + (i * 53) % 9000) for i in range(1200)]
+    _run(2048, rows, seed=8)
