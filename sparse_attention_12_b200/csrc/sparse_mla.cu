@@ -12,7 +12,7 @@
 //   S-CTA (rank 0): S = Q C^T and the softmax.
 //     * Q (128 heads x 576 bf16): dims 0..511 in TMEM as the A operand (256 columns), the 64 rope
 //       dims in shared memory (one 128-byte-swizzled block).
-//     * 20 producer warps gather latent dims 0..511 of the selected rows with 16-byte cp.async (8
+//     * 8 producer warps gather latent dims 0..511 of the selected rows with 16-byte cp.async (8
 //       lanes per 128-byte row segment, XOR-swizzled on the way into the canonical 128-byte-swizzled
 //       K-major UMMA layout) into an 8-slot ring (slot = 64-dim block of the current tile); a ninth
 //       warp fetches the rope dims 512..575 with TMA gather4 (4 rows per copy) into a 2-slot ring.
@@ -27,7 +27,7 @@
 //       bytes complete the O-CTA's barrier for that P buffer (two buffers, alternating by tile).
 //   O-CTA (rank 1): O = P V.
 //     * O (128 heads x 512 fp32) fills its whole TMEM. V = c[0:512] of the same rows (mostly L2
-//       hits: the S-CTA fetched them) is gathered by 20 producer warps in units of 128 keys x 128
+//       hits: the S-CTA fetched them) is gathered by 8 producer warps in units of 128 keys x 128
 //       dims (4 per tile).
 //     * Per tile: 32 tcgen05.mma (M=128, N=128 dims, K=16 keys), A = P (shared memory, K-major),
 //       B = V (MN-major). Completion is multicast back to the S-CTA to free the P buffer.
@@ -62,17 +62,17 @@ constexpr int kBlk = kTile * 128;            // 128 keys x 64 dims bf16 = 16 KB
 constexpr int kKSlots = 8;                   // S-CTA cp.async ring: latent blocks 0..7 of a tile, slot = block
 constexpr int kRSlots = 2;                   // S-CTA TMA ring: the rope block (dims 512..575) of a tile
 constexpr int kVSlots = 4;                   // O-CTA ring slots (two 64-dim blocks of one tile each)
-constexpr int kProdWarps = 20;               // warps 0..19: cp.async gather producers
+constexpr int kProdWarps = 8;                // warps 0..7: cp.async gather producers
 // A producer group fills one ring unit at a time; each ring slot belongs to exactly one group
 // (slot % groups == group), so a group never runs two uses ahead of the consumer on a slot's
 // barrier, which a parity wait could not tell from one use ahead.
-constexpr int kSGroupWarps = 5, kSGroups = kProdWarps / kSGroupWarps;  // S-CTA: 4 groups, 8 slots
-constexpr int kOGroupWarps = 5, kOGroups = kProdWarps / kOGroupWarps;  // O-CTA: 4 groups, 4 slots
-constexpr int kMmaWarp = kProdWarps;         // warp 20: TMEM allocator and MMA issuer
-constexpr int kSoftWarp0 = kProdWarps + 1;   // warps 21..28: softmax (S-CTA) / correction (O-CTA),
+constexpr int kSGroupWarps = 2, kSGroups = kProdWarps / kSGroupWarps;  // S-CTA: 4 groups, 8 slots
+constexpr int kOGroupWarps = 2, kOGroups = kProdWarps / kOGroupWarps;  // O-CTA: 4 groups, 4 slots
+constexpr int kMmaWarp = kProdWarps;         // warp 8: TMEM allocator and MMA issuer
+constexpr int kSoftWarp0 = kProdWarps + 1;   // warps 9..16: softmax (S-CTA) / correction (O-CTA),
 constexpr int kSoftWarps = 8;                //   two per TMEM lane quadrant
 constexpr int kSubs = kSoftWarps / 4;        // column halves per quadrant
-constexpr int kRopeWarp = kSoftWarp0 + kSoftWarps;  // warp 29: rope blocks by TMA gather4 (S-CTA only)
+constexpr int kRopeWarp = kSoftWarp0 + kSoftWarps;  // warp 17: rope blocks by TMA gather4 (S-CTA only)
 constexpr int kThreads = 32 * (kRopeWarp + 1);
 constexpr int kRowIters = (kMaxKeysPerCta + kThreads - 1) / kThreads;
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
@@ -389,7 +389,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           mbar_drain(&bar[B_RFULL + i % kRSlots], (i / kRSlots) & 1, p.status);
       __syncwarp();
     } else {
-      // ---------- S-CTA softmax (warps 21..28: thread = head h, keys 64*sub .. 64*sub+63) ----------
+      // ---------- S-CTA softmax (warps 9..16: thread = head h, keys 64*sub .. 64*sub+63) ----------
       float* red = reinterpret_cast<float*>(base + Smem::kRed);    // [2][kSubs][128]
       float* redl = reinterpret_cast<float*>(base + Smem::kRedL);  // [2][kSubs][128]: l, lr
       const uint32_t peer_p = peer_addr(smem_u32(base + Smem::kP), 1);
@@ -586,7 +586,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     } else if (warp < kSoftWarp0 + kSoftWarps) {
-      // ---------- O-CTA correction + epilogue (warps 21..28: head h, O columns 256*sub .. +255) ------
+      // ---------- O-CTA correction + epilogue (warps 9..16: head h, O columns 256*sub .. +255) ------
       const volatile float* stats = reinterpret_cast<const volatile float*>(base + Smem::kStats);
       const uint32_t ocol = tmem + lane_base + kColO + 256 * sub;
       bool ok = true;
