@@ -257,15 +257,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t t_row = tmem_base + lane_base + static_cast<uint32_t>(a * p.ncols);
         for (int q = (half + it * m) & 1; q < m; q += 2) {  // (tile, query) items alternate between the two warps
           const float4* w4 = reinterpret_cast<const float4*>(g_w + q * NHI);
-          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+          float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);  // four chains: the head sum is latency-bound
           auto accumulate = [&](const uint32_t* v, int nv, int w0) {
 #pragma unroll
             for (int i = 0; i < nv / 4; ++i) {
               const float4 ww = w4[w0 / 4 + i];
-              a0 = fmaf(ww.x, fmaxf(__uint_as_float(v[4 * i + 0]), 0.f), a0);
-              a1 = fmaf(ww.y, fmaxf(__uint_as_float(v[4 * i + 1]), 0.f), a1);
-              a2 = fmaf(ww.z, fmaxf(__uint_as_float(v[4 * i + 2]), 0.f), a2);
-              a3 = fmaf(ww.w, fmaxf(__uint_as_float(v[4 * i + 3]), 0.f), a3);
+              // chains (a0, a1) and (a2, a3) advance in pairs: one instruction per two heads
+              a01 = fma_f32x2(make_float2(fmaxf(__uint_as_float(v[4 * i + 0]), 0.f), fmaxf(__uint_as_float(v[4 * i + 1]), 0.f)),
+                              make_float2(ww.x, ww.y), a01);
+              a23 = fma_f32x2(make_float2(fmaxf(__uint_as_float(v[4 * i + 2]), 0.f), fmaxf(__uint_as_float(v[4 * i + 3]), 0.f)),
+                              make_float2(ww.z, ww.w), a23);
             }
           };
           if constexpr (NHI % 32 == 0) {
@@ -282,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_ld();
             accumulate(v, 16, 0);
           }
-          const float score = ((a0 + a1) + (a2 + a3)) * g_sq[q] * sk;
+          const float score = ((a01.x + a01.y) + (a23.x + a23.y)) * g_sq[q] * sk;
           cache[q * p.slice_cap + jl] = sel::order_key(score);  // positions past the query are never read
         }
         tc_fence_before();

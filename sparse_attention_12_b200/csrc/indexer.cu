@@ -25,6 +25,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include <cmath>
 
 #include "dsa_internal.h"
@@ -359,38 +361,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float sk = (j <= p_last) ? g_scale[c * kIdxTileKeys + quad * 32 + lane] : 0.f;
         tc_fence_after();
         const uint32_t t_row = tmem_base + lane_base + static_cast<uint32_t>(a * p.ncols);
-        // items (tile it, query q) alternate between the quadrant's two warps
-        for (int q = (half + it * gm.nq) & 1; q < gm.nq; q += 2) {
-          const float4* w4 = reinterpret_cast<const float4*>(g_w + qb * kIdxCols + q * NHI);
-          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;  // four chains: the head sum is latency-bound
-          auto accumulate = [&](const uint32_t* v, int nv, int w0) {
+        // items (tile it, query q) alternate between the quadrant's two warps; a warp takes its
+        // items two at a time (q and q + 2) when it has two, so that eight independent chains hide
+        // the latency of the head sum. Per item the arithmetic and its order are the same.
+        auto items = [&](auto two_tag, int qa) {
+          constexpr bool kTwo = decltype(two_tag)::value;
+          const int qz = kTwo ? qa + 2 : qa;
+          const float4* wa = reinterpret_cast<const float4*>(g_w + qb * kIdxCols + qa * NHI);
+          const float4* wz = reinterpret_cast<const float4*>(g_w + qb * kIdxCols + qz * NHI);
+          // chains (a0, a1) and (a2, a3) of each item advance in pairs: one instruction per two heads
+          float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
+          float2 z01 = make_float2(0.f, 0.f), z23 = make_float2(0.f, 0.f);
+          auto accumulate = [&](const uint32_t* v, const float4* w4, int nv, int w0, float2& x01, float2& x23) {
 #pragma unroll
             for (int i = 0; i < nv / 4; ++i) {
               const float4 ww = w4[w0 / 4 + i];
-              a0 = fmaf(ww.x, fmaxf(__uint_as_float(v[4 * i + 0]), 0.f), a0);
-              a1 = fmaf(ww.y, fmaxf(__uint_as_float(v[4 * i + 1]), 0.f), a1);
-              a2 = fmaf(ww.z, fmaxf(__uint_as_float(v[4 * i + 2]), 0.f), a2);
-              a3 = fmaf(ww.w, fmaxf(__uint_as_float(v[4 * i + 3]), 0.f), a3);
+              x01 = fma_f32x2(make_float2(fmaxf(__uint_as_float(v[4 * i + 0]), 0.f), fmaxf(__uint_as_float(v[4 * i + 1]), 0.f)),
+                              make_float2(ww.x, ww.y), x01);
+              x23 = fma_f32x2(make_float2(fmaxf(__uint_as_float(v[4 * i + 2]), 0.f), fmaxf(__uint_as_float(v[4 * i + 3]), 0.f)),
+                              make_float2(ww.z, ww.w), x23);
             }
           };
           if constexpr (NHI % 32 == 0) {
 #pragma unroll
-            for (int c = 0; c < NHI / 32; ++c) {
-              uint32_t v[32];
-              tmem_ld32(t_row + static_cast<uint32_t>(q * NHI + c * 32), v);
+            for (int cc = 0; cc < NHI / 32; ++cc) {
+              uint32_t va[32], vz[32];
+              tmem_ld32(t_row + static_cast<uint32_t>(qa * NHI + cc * 32), va);
+              if constexpr (kTwo) tmem_ld32(t_row + static_cast<uint32_t>(qz * NHI + cc * 32), vz);
               tmem_wait_ld();
-              accumulate(v, 32, c * 32);
+              accumulate(va, wa, 32, cc * 32, a01, a23);
+              if constexpr (kTwo) accumulate(vz, wz, 32, cc * 32, z01, z23);
             }
           } else {
-            uint32_t v[16];
-            tmem_ld16(t_row + static_cast<uint32_t>(q * NHI), v);
+            uint32_t va[16], vz[16];
+            tmem_ld16(t_row + static_cast<uint32_t>(qa * NHI), va);
+            if constexpr (kTwo) tmem_ld16(t_row + static_cast<uint32_t>(qz * NHI), vz);
             tmem_wait_ld();
-            accumulate(v, 16, 0);
+            accumulate(va, wa, 16, 0, a01, a23);
+            if constexpr (kTwo) accumulate(vz, wz, 16, 0, z01, z23);
           }
-          const float acc = (a0 + a1) + (a2 + a3);
-          float score = acc * g_sq[qb * 16 + q] * sk;
-          if (j > gm.pos0 + q) score = -INFINITY;
-          if (j < p.ld) p.scores[static_cast<int64_t>(gm.row0 + q) * p.ld + j] = score;
+          auto store = [&](int q, float2 x01, float2 x23) {
+            const float acc = (x01.x + x01.y) + (x23.x + x23.y);
+            float score = acc * g_sq[qb * 16 + q] * sk;
+            if (j > gm.pos0 + q) score = -INFINITY;
+            if (j < p.ld) p.scores[static_cast<int64_t>(gm.row0 + q) * p.ld + j] = score;
+          };
+          store(qa, a01, a23);
+          if constexpr (kTwo) store(qz, z01, z23);
+        };
+        for (int q = (half + it * gm.nq) & 1; q < gm.nq; q += 4) {
+          if (q + 2 < gm.nq)
+            items(std::true_type{}, q);
+          else
+            items(std::false_type{}, q);
         }
         tc_fence_before();
         __syncwarp();

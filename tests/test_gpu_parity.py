@@ -99,6 +99,14 @@ def test_k_equals_visible_positions():
     run_all_checks(wl)
 
 
+def test_prefill_two_splits_with_empty_units():
+    # k = 4096 needs two units per query row (2048 entries each); rows before position 2048 have an
+    # empty second unit, so the persistent clusters meet units without tiles between full ones
+    wl = synth.custom("split_prefill", [2300], [2300], n_heads_index=16, topk=4096, n_heads=16,
+                      needles="prefill", n_needles=4)
+    run_all_checks(wl)
+
+
 # ---------------------------------------------------------------------------------------------
 # the workload shapes
 
