@@ -95,6 +95,21 @@ def test_masked_mha_128_heads():
     _run([300, 77], H=128, topk=128, seed=6)
 
 
+def test_masked_mha_ragged_many_heads():
+    """64 heads over ragged requests (a partial last tile, a request of 1000 positions over eight
+    query tiles, a request just past one tile); sparse sets (k = 300), rows sampled in every tile
+    and at every tile edge."""
+    lens = [600, 1000, 130]
+    T = sum(lens)
+    rows = sorted(set(list(range(0, T, 7)) + [127, 128, 255, 256, 599, 600, 727, 728, 855, 856, 1599, 1600, T - 1]))
+    _run(lens, H=64, topk=300, seed=7, rows=rows)
+
+
+def test_masked_mha_many_heads_dense_sets():
+    """96 heads with k above every prefix: plain causal multi-head attention."""
+    _run([520, 256], H=96, topk=1024, seed=8, rows=list(range(0, 776, 5)) + [255, 256, 511, 519, 775])
+
+
 def test_masked_mha_rejects_requests_with_a_cached_prefix():
     """n_b != m_b is not a whole prefill: the kernel records DSA_ERR_DEVICE_INDEX and writes nothing."""
     lens, qs = [200], [100]
@@ -110,3 +125,22 @@ def test_masked_mha_rejects_requests_with_a_cached_prefix():
     dsa.masked_mha(batch, plan, q, k, v, S, wl.softmax_scale, out=out)
     assert dsa.status_read(plan) == 6
     assert bool((out == 7.0).all())
+
+
+def test_masked_mha_rejects_a_cached_prefix_beside_a_whole_prefill():
+    """128 heads, a cached-prefix request next to a whole prefill: the first is reported and left
+    unwritten, the second computed."""
+    lens, qs = [200, 300], [100, 300]
+    wl = synth.custom("mha_bad2", lens, lens, n_heads=128, topk=64)
+    x = synth.make_mha_inputs(wl, seed=9)
+    batch, _ = _batch(lens, qs)
+    plan = dsa.plan(batch, 16)
+    S = torch.from_numpy(synth.random_index_sets(lens, qs, 64, seed=9)).cuda()
+    sel = torch.cat([torch.arange(100, 200), torch.arange(200, 500)]).cuda()  # rows of the queries
+    q = _bf16(x.q).index_select(0, sel).contiguous()
+    k = _bf16(x.k).index_select(0, sel).contiguous()
+    v = _bf16(x.v).index_select(0, sel).contiguous()
+    out = torch.full((400, 128, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    dsa.masked_mha(batch, plan, q, k, v, S, wl.softmax_scale, out=out)
+    assert dsa.status_read(plan) == 6
+    assert bool((out[:100] == 7.0).all())
