@@ -604,9 +604,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             uint32_t v[32];
             tmem_ld32_sync(srow + 32 * c, v);
             const uint32_t m = msk[4 * i + 2 * sub + c];
+            if (m == 0xFFFFFFFFu) {  // every key of the chunk selected (the usual case; warp-uniform)
+              // the scale is positive and rounding is monotonic: max(v) * s == max(v * s)
+              float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if ((m >> j) & 1u) pmax = fmaxf(pmax, __uint_as_float(v[j]) * p.scale_log2);
+              for (int j = 0; j < 32; ++j) mx[j & 3] = fmaxf(mx[j & 3], __uint_as_float(v[j]));
+              pmax = fmaxf(pmax, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if ((m >> j) & 1u) pmax = fmaxf(pmax, __uint_as_float(v[j]) * p.scale_log2);
+            }
           }
           // tile maximum of head h across this quadrant's warps (shared memory + mbarrier)
           red[(sb * kSubs + sub) * 128 + h] = pmax;
