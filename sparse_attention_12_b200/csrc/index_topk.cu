@@ -218,11 +218,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = mbar_wait(qfull, 0, p.status, kDevErrTimeout);
         const uint32_t idesc = umma_idesc(128, static_cast<uint32_t>(m * NHI), 0, 0, 0);
         const uint64_t bd = umma_desc_sw128(smem_u32(qbuf), 16, 1024);
+        int s = 0, s_par = 0, a = 0, a_par = 1;  // key stage and accumulator of tile it, parities to wait for
         for (int it = 0; it < nt && ok; ++it) {
-          const int s = it % p.nstages;
-          const int a = it % p.nacc;
-          ok = mbar_wait(&kfull[s], (it / p.nstages) & 1, p.status, kDevErrTimeout) &&
-               mbar_wait(&tempty[a], ((it / p.nacc) & 1) ^ 1, p.status, kDevErrTimeout);
+          ok = mbar_wait(&kfull[s], s_par, p.status, kDevErrTimeout) &&
+               mbar_wait(&tempty[a], a_par, p.status, kDevErrTimeout);
           if (!ok) break;
           tc_fence_after();
           const uint64_t ad = umma_desc_sw128(smem_u32(ring + s * kStageBytes), 16, 1024);
@@ -232,6 +231,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_f8_ss(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, kk > 0 ? 1u : 0u);
           mma_commit(&kempty[s]);
           mma_commit(&tfull[a]);
+          if (++s == p.nstages) s = 0, s_par ^= 1;
+          if (++a == p.nacc) a = 0, a_par ^= 1;
         }
         // every MMA this thread issued has completed before TMEM is freed (also after an error)
         mma_commit(mdone);
@@ -245,11 +246,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int half = ew >> 2;
       const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
       bool ok = true;
-      for (int it = 0; it < nt && ok; ++it) {
+      int a = 0, a_par = 0;  // accumulator of tile it and the parity to wait for
+      for (int it = 0; it < nt && ok; ++it, (++a == p.nacc) ? (a = 0, a_par ^= 1) : 0) {
         const int c = it % kScaleSlots;
-        const int a = it % p.nacc;
         ok = __all_sync(0xffffffffu, mbar_wait(&sfull[c], (it / kScaleSlots) & 1, p.status, kDevErrTimeout) &&
-                                         mbar_wait(&tfull[a], (it / p.nacc) & 1, p.status, kDevErrTimeout));
+                                         mbar_wait(&tfull[a], a_par, p.status, kDevErrTimeout));
         if (!ok) break;
         const int jl = it * kIdxTileKeys + quad * 32 + lane;  // key index within this CTA's slice
         const float sk = (kbase + jl <= p_last) ? g_scale[c * kIdxTileKeys + quad * 32 + lane] : 0.f;

@@ -284,27 +284,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
       // ---------------- MMA issuer ----------------
       if (lane == 0) {
+        // the group bounds and sizes come one group ahead, so a group switch waits on no load
         int g = g_first;
         int gend = __ldg(p.grp_tile0 + g + 1);
-        int nq = 0, qcount = 0, qb = 0;
+        int nq = __ldg(p.grp_nq + g);
+        int g_last = (g + 1 < G) ? g + 1 : g;
+        int gend_next = __ldg(p.grp_tile0 + g_last + 1), nq_next = __ldg(p.grp_nq + g_last);
+        int qcount = 0, qb = 0;
+        int s = 0, s_par = 0, a = 0, a_par = 1;  // key stage and accumulator of tile it, parities to wait for
         bool ok = true;
         for (int u = u0, it = 0; u < u1 && ok; ++u, ++it) {
           const bool newg = (u == u0) || (u == gend);
           if (u == gend) {
             ++g;
-            gend = __ldg(p.grp_tile0 + g + 1);
+            gend = gend_next;
+            nq = nq_next;
+            g_last = (g + 1 < G) ? g + 1 : g;
+            gend_next = __ldg(p.grp_tile0 + g_last + 1);
+            nq_next = __ldg(p.grp_nq + g_last);
           }
           if (newg) {
             qb = qcount & 1;
             ok = mbar_wait(&qfull[qb], (qcount >> 1) & 1, p.status, kDevErrTimeout);
             if (!ok) break;
-            nq = __ldg(p.grp_nq + g);
             ++qcount;
           }
-          const int s = it % p.nstages;
-          const int a = it % p.nacc;
-          ok = mbar_wait(&kfull[s], (it / p.nstages) & 1, p.status, kDevErrTimeout) &&
-               mbar_wait(&tempty[a], ((it / p.nacc) & 1) ^ 1, p.status, kDevErrTimeout);
+          ok = mbar_wait(&kfull[s], s_par, p.status, kDevErrTimeout) &&
+               mbar_wait(&tempty[a], a_par, p.status, kDevErrTimeout);
           if (!ok) break;
           tc_fence_after();
           const uint32_t idesc = umma_idesc(128, static_cast<uint32_t>(nq * NHI), 0, 0, 0);
@@ -318,6 +324,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&kempty[s]);
           mma_commit(&tfull[a]);
           if (u + 1 == gend || u + 1 == u1) mma_commit(&qempty[qb]);
+          if (++s == p.nstages) s = 0, s_par ^= 1;
+          if (++a == p.nacc) a = 0, a_par ^= 1;
         }
         // every MMA this thread issued has completed before TMEM is freed (also after an error)
         mma_commit(mdone);
@@ -332,7 +340,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
       int g = g_first;
       int gstart = __ldg(p.grp_tile0 + g), gend = __ldg(p.grp_tile0 + g + 1);
+      int gend_next = __ldg(p.grp_tile0 + min(g + 1, G - 1) + 1);  // one group ahead
       int qcount = 0, qb = 0;
+      int a = 0, a_par = 0;  // accumulator of tile it and the parity to wait for
       GroupMeta gm{};
       bool ok = true;
       for (int u = u0, it = 0; u < u1 && ok; ++u, ++it) {
@@ -340,7 +350,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u == gend) {
           ++g;
           gstart = gend;
-          gend = __ldg(p.grp_tile0 + g + 1);
+          gend = gend_next;
+          gend_next = __ldg(p.grp_tile0 + min(g + 1, G - 1) + 1);
         }
         if (newg) {
           qb = qcount & 1;
@@ -353,10 +364,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int j = kt * kIdxTileKeys + quad * 32 + lane;
         const int p_last = gm.pos0 + gm.nq - 1;
         const int c = it % kScaleSlots;
-        const int a = it % p.nacc;
         // (not kfull: key stages recycle at MMA completion and may run a whole ring ahead of here)
         ok = __all_sync(0xffffffffu, mbar_wait(&sfull[c], (it / kScaleSlots) & 1, p.status, kDevErrTimeout) &&
-                                         mbar_wait(&tfull[a], (it / p.nacc) & 1, p.status, kDevErrTimeout));
+                                         mbar_wait(&tfull[a], a_par, p.status, kDevErrTimeout));
         if (!ok) break;
         const float sk = (j <= p_last) ? g_scale[c * kIdxTileKeys + quad * 32 + lane] : 0.f;
         tc_fence_after();
@@ -422,6 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(&tempty[a]);
           if (u + 1 == gend || u + 1 == u1) mbar_arrive(&qempty[qb]);
         }
+        if (++a == p.nacc) a = 0, a_par ^= 1;
       }
     }
   }
