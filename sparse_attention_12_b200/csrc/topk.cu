@@ -133,7 +133,11 @@ __global__ void __launch_bounds__(NT) topk_kernel(const int32_t* __restrict__ ro
   const int64_t key_off = static_cast<int64_t>(gridDim.x / (kMerge ? 1 : nsl_max)) * nsl_max * kpad;
   const int32_t* cands = cand_ws + static_cast<int64_t>(t) * nsl_max * kpad;
   const uint32_t* cand_keys = reinterpret_cast<const uint32_t*>(cands + key_off);
-  auto position = [&](int i) -> int { return kMerge ? __ldg(cands + (i / k) * kpad + i % k) : base + i; };
+  // candidate i of the merge sits at slice i / k, entry i % k (rows of kpad entries; kpad == k for
+  // k a multiple of 4, where the index is i itself)
+  const bool packed = kpad == k;
+  auto cand_at = [&](int i) -> int { return packed ? i : (i / k) * kpad + i % k; };
+  auto position = [&](int i) -> int { return kMerge ? __ldg(cands + cand_at(i)) : base + i; };
   const bool to_cands = !kMerge && nsl > 1;
   int32_t* out = to_cands ? cand_ws + (static_cast<int64_t>(t) * nsl_max + sl) * kpad : S + static_cast<int64_t>(t) * k;
   uint32_t* out_key = to_cands ? reinterpret_cast<uint32_t*>(out + key_off) : nullptr;
@@ -178,7 +182,7 @@ __global__ void __launch_bounds__(NT) topk_kernel(const int32_t* __restrict__ ro
           float v[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            if (e < nv[g]) v[e] = key_value(__ldg(cand_keys + ((j0 + e) / k) * kpad + (j0 + e) % k));
+            if (e < nv[g]) v[e] = key_value(__ldg(cand_keys + cand_at(j0 + e)));
           f[g] = make_float4(v[0], v[1], v[2], v[3]);
         } else {  // base + j0 + 3 < ld: base and j0 are multiples of 4, ld % 4 == 0, base + j0 < L <= ld
           f[g] = __ldg(reinterpret_cast<const float4*>(row + base + j0));
