@@ -49,6 +49,14 @@ BatchDev to_dev(const dsa_batch_t* b) {
 
 dsa_status_t from_cuda(int e) { return e == 0 ? DSA_OK : DSA_ERR_CUDA; }
 
+// The sparse MLA step: keys on the MMA's M axis for a few heads, heads on it otherwise.
+int launch_mla(const BatchDev& b, const void* plan, const void* q, int H, const void* kv_cache, const int32_t* S,
+               int k, float softmax_scale, void* out, float* lse, void* ws, void* stream) {
+  if (H <= kNarrowHeads)
+    return launch_sparse_mla_narrow(b, plan, q, H, kv_cache, S, k, softmax_scale, out, lse, ws, stream);
+  return launch_sparse_mla(b, plan, q, H, kv_cache, S, k, softmax_scale, out, lse, ws, stream);
+}
+
 size_t scores_ld(const dsa_batch_t* b) {
   return (static_cast<size_t>(b->max_seq_len) + 127) / 128 * 128;
 }
@@ -195,7 +203,7 @@ dsa_status_t dsa_sparse_mla(const dsa_batch_t* batch, const void* plan, const vo
   const size_t need = sparse_mla_ws_bytes(batch->total_q, H, k);
   if (need > 0 && (!ws || !aligned16(ws))) return DSA_ERR_INVALID_ARG;
   if (ws_bytes < need) return DSA_ERR_WORKSPACE;
-  return from_cuda(launch_sparse_mla(to_dev(batch), plan, q, H, kv_cache, S, k, softmax_scale, out, lse, ws, stream));
+  return from_cuda(launch_mla(to_dev(batch), plan, q, H, kv_cache, S, k, softmax_scale, out, lse, ws, stream));
 }
 
 dsa_status_t dsa_cache_write(const dsa_batch_t* batch, const void* plan, const float* k_new, const void* c_new,
@@ -272,7 +280,7 @@ dsa_status_t dsa_layer(const dsa_batch_t* batch, const uint8_t* qI, const float*
   int e = launch_plan(bd, nhI, plan, stream);
   if (!e) e = launch_index_scores(bd, plan, qI, qI_scale, wI, nhI, kI_cache, kI_scale, scores, ld, stream);
   if (!e) e = launch_topk(bd, plan, scores, ld, k, S, mla_ws, stream);
-  if (!e) e = launch_sparse_mla(bd, plan, q, H, kv_cache, S, k, softmax_scale, out, lse, mla_ws, stream);
+  if (!e) e = launch_mla(bd, plan, q, H, kv_cache, S, k, softmax_scale, out, lse, mla_ws, stream);
   return from_cuda(e);
 }
 

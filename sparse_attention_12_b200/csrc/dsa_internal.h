@@ -124,6 +124,12 @@ size_t sparse_mla_ws_bytes(int T, int H, int k);
 int sparse_mla_splits(int T, int k);
 int launch_sparse_mla(const BatchDev& b, const void* plan, const void* q, int H, const void* kv_cache,
                       const int32_t* S, int k, float softmax_scale, void* out, float* lse, void* ws, void* stream);
+// Head counts up to kNarrowHeads run the keys-on-M kernel (sparse_mla_narrow.cu), with the same
+// splits and workspace as launch_sparse_mla.
+constexpr int kNarrowHeads = 16;
+int launch_sparse_mla_narrow(const BatchDev& b, const void* plan, const void* q, int H, const void* kv_cache,
+                             const int32_t* S, int k, float softmax_scale, void* out, float* lse, void* ws,
+                             void* stream);
 constexpr int kMaxMhaSeqLen = 65536;  // longest request the masked MHA mode takes
 size_t masked_mha_ws_bytes(int T, int max_seq_len);
 int launch_masked_mha(const BatchDev& b, const void* plan, const void* q, const void* k, const void* v, int H,
