@@ -14,6 +14,11 @@
 //   O^T[dim, h] += V^T P^T      M = 128 dims (four of them), K = 128 keys: 8 MMAs each
 // so every accumulator row is a real key or a real value dimension; S^T and O^T take 160 TMEM
 // columns and one CTA (one SM) runs the whole of a unit (query row, split of S_t).
+// Measured on B200: a tcgen05.mma of N <= 32 costs ~46 cycles whether M is 64 or 128 (64 cycles at
+// N = 128, 128 at N = 256), so a tile's 68 MMAs take ~1.6 us. The tile period (~4.7 us) is set by
+// the ring instead: a tile's V slots stay until its P V MMAs complete, so the next tile's last
+// three slots are gathered only after the softmax and the products of this one. (Tiles of 64 keys
+// with a 2.5-tile ring, and two softmax groups on alternating tiles, were measured slower.)
 //
 // Persistent CTAs, one per SM, each taking the units u = cta, cta + ctas, ... in turn:
 //   * warps 0..7 gather the rows of each tile of 128 keys with 16-byte cp.async (8 lanes per
