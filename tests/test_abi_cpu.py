@@ -148,6 +148,14 @@ def test_topk_and_mla_validation(lib):
     need = lib.dsa_sparse_mla_workspace_size(ctypes.byref(b), 128, 2048)
     assert need > 0          # 3 rows cannot fill the GPU: split partials need workspace
     assert mla(ws_bytes=need - 1) == 3
+    # 16 heads or fewer run the few-head kernel: the same splits and partial-output layout
+    # ([T][splits][H][512] fp32, then [T][splits][H] log-sum-exp), so the same size formula
+    splits = min(74 // 3, 16, 2048 // 128)
+    a16 = lambda x: (x + 15) // 16 * 16
+    for H in (16, 5, 1):
+        need_h = lib.dsa_sparse_mla_workspace_size(ctypes.byref(b), H, 2048)
+        assert need_h == a16(4 * 3 * splits * H * 512) + a16(4 * 3 * splits * H)
+        assert mla(H=H, ws_bytes=need_h - 1) == 3
 
 
 @no_gpu
